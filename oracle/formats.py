@@ -75,7 +75,10 @@ def _nearest_sorted(vals: np.ndarray, x: np.ndarray) -> np.ndarray:
     d_lo = np.abs(x - vals[lo])
     d_hi = np.abs(vals[hi] - x)
     pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
-    return np.where(pick_hi, hi, lo)
+    idx = np.where(pick_hi, hi, lo)
+    # saturation, stated directly: far beyond the table the binary64 distances to the last
+    # two entries can round to the same value
+    return np.where(x >= vals[-1], len(vals) - 1, idx)
 
 
 def round_elem(x32: np.ndarray, fmt: Format):

@@ -140,6 +140,16 @@ def test_e2m1_round_brute_force(kind):
     assert np.all(np.signbit(got) == np.signbit(x))
 
 
+@pytest.mark.parametrize("kind", ["MXFP4", "MXINT4"])
+def test_element_rounding_saturates_for_huge_inputs(kind):
+    fmt = F.make_format(kind)
+    x = np.float32([1e6, 7.3e16, 1e30, 3.4e38, -7.3e16, -3.4e38])
+    _, q = F.round_elem(x, fmt)
+    top = fmt.qmax
+    assert q.tolist() == [top] * 4 + [-top, -top]
+    assert F.E4M3_POS[F.e4m3_nearest_code(np.float32([7.3e16, 3.4e38]))].tolist() == [448.0] * 2
+
+
 def test_e2m1_documented_ties():
     fmt = F.make_format("MXFP4")
     x = np.float32([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.5, -0.25, -5.0])
