@@ -1,0 +1,420 @@
+"""Benchmark of the DualQuant hot path on B200.
+
+One step = one full-model dual-scale solve of the Llama-3.1-8B-shaped layer set (32 blocks x
+q/k/v/o/gate/up/down, 6.98e9 bf16 weights, NVFP4, 16 BCD iterations) through
+dq_solve_batched, followed by the activation rescale + NVFP4 quantization of an 8192 x 4096
+activation with the column scales of that step's block-0 k_proj (dq_act_quant).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank solves its own layer set
+(different seeds), no collective on the data path; timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "BCD weight elems×iters/s and full-model solve s; % of B200 HBM roofline"
+UNIT = "elem*iter/s"
+CFG_ID = 3
+# FP32 operations per element and BCD iteration in the formulation (FMA counted once):
+# Q-step 2 mul + 1 rounding; r-step q*c, W*qc, (qc)^2; c-step q*r, W*qr, (qr)^2.
+OPS_PER_ELEM_ITER = 9
+# iteration 0 (initialisation): |W| max, Q-step (3), c-step sums (3), W^2
+OPS_PER_ELEM_INIT = 8
+# algorithmic bytes per element and iteration of a per-iteration streaming solve (read W
+# in bf16 + NVFP4 scale state read and write): the HBM-equivalent figure
+HBM_BYTES_PER_ELEM_ITER = 2.125
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--blocks", type=int, default=None,
+                    help="solve only the first B blocks (profiling runs; not a bench value)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------- CPU oracle
+def cpu_sample_solve(W: np.ndarray, amax: float, iters: int):
+    """Oracle solve of a bounded sample; returns (elem*iter/s, seconds, elements)."""
+    from oracle import formats as F
+    from oracle import solver as S
+    t0 = time.perf_counter()
+    S.solve(W, F.make_format("NVFP4"), iters, amax=amax)
+    dt = time.perf_counter() - t0
+    return W.size * iters / dt, dt, W.size
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    cfg = wl.CONFIGS[CFG_ID]
+    Wk = wl.weight_host(cfg, 0, 1).float().numpy().astype(np.float64)     # block-0 k_proj
+    amax = float(np.max(np.abs(Wk)))
+    sample = Wk[:, :1024]
+    desc = "block-0 k_proj of the 8B layer set, columns 0..1023 (1024x1024), 16 iterations"
+    for _ in range(args.warmup):
+        cpu_sample_solve(sample, amax, cfg.iters)
+    times = []
+    for _ in range(args.steps):
+        _, dt, _ = cpu_sample_solve(sample, amax, cfg.iters)
+        times.append(dt)
+    tot = sum(times)
+    value = sample.size * cfg.iters * args.steps / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "oracle sample: " + desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our path
+def run_ours(args, world, rank, local):
+    import calibration_free_dual_b200 as dq
+    from calibration_free_dual_b200 import _lib
+
+    dev = torch.device("cuda", local)
+    cfg = wl.CONFIGS[CFG_ID]
+    layer = cfg.layer_set()
+    if args.blocks is not None:
+        layer = [e for e in layer if e[0] < args.blocks]
+    T = cfg.iters
+    fmt = dq.fmt_of(cfg.fmt)
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs (device-generated, seeded per rank) and preallocated outputs
+    Ws = [wl.weight_device(cfg, b, p, device=dev, seed_offset=rank) for b, p, _, _ in layer]
+    X = wl.act_device(device=dev)
+    outs = [dq.api.solve_outputs(W.shape[0], W.shape[1], fmt, T, dev) for W in Ws]
+    count = len(Ws)
+    ms = (ctypes.c_int64 * count)(*[W.shape[0] for W in Ws])
+    ns = (ctypes.c_int64 * count)(*[W.shape[1] for W in Ws])
+    lib = _lib.get()
+    ws_bytes = lib.dq_solve_workspace_bytes(count, ms, ns, fmt, T)
+    ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
+    act_out = dict(x_packed=torch.empty((X.shape[0], X.shape[1] // 2), dtype=torch.uint8,
+                                        device=dev),
+                   scales=torch.empty((X.shape[0], X.shape[1] // 16), dtype=torch.uint8,
+                                      device=dev),
+                   tensor_scale=torch.empty((1,), dtype=torch.float32, device=dev))
+    act_ws = torch.empty((256,), dtype=torch.uint8, device=dev)
+    k0 = next(i for i, (b, p, _, _) in enumerate(layer) if b == 0 and p == 1)
+
+    def mats_for(Wlist):
+        arr = (_lib.dq_matrix * count)()
+        for i, (W, o) in enumerate(zip(Wlist, outs)):
+            arr[i] = _lib.dq_matrix(W.data_ptr(), W.shape[0], W.shape[1], W.stride(0), None,
+                                    None, o["q_packed"].data_ptr(), o["r"].data_ptr(),
+                                    o["c"].data_ptr(), o["block_scales"].data_ptr(),
+                                    o["tensor_scale"].data_ptr(), o["mse"].data_ptr())
+        return arr
+
+    mats = mats_for(Ws)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+
+    def step(mats_arr, Xin):
+        st = lib.dq_solve_batched(mats_arr, count, _lib.DQ_BF16, fmt, T,
+                                  ctypes.c_void_p(ws.data_ptr()), ws_bytes, sptr)
+        if st != 0:
+            raise dq.DQError(st, "dq_solve_batched")
+        st = lib.dq_act_quant(ctypes.c_void_p(Xin.data_ptr()), _lib.DQ_BF16, Xin.shape[0],
+                              Xin.shape[1], Xin.stride(0),
+                              ctypes.c_void_p(outs[k0]["c"].data_ptr()), fmt,
+                              ctypes.c_void_p(act_out["x_packed"].data_ptr()),
+                              ctypes.c_void_p(act_out["scales"].data_ptr()),
+                              ctypes.c_void_p(act_out["tensor_scale"].data_ptr()),
+                              ctypes.c_void_p(act_ws.data_ptr()), act_ws.numel(), sptr)
+        if st != 0:
+            raise dq.DQError(st, "dq_act_quant")
+
+    elems = sum(W.numel() for W in Ws)
+    for _ in range(args.warmup):
+        step(mats, X)
+    torch.cuda.synchronize(dev)
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # per-launch events for the solve kernel over the timed region
+    per_step = sum((n + 31) // 32 for n in _group_sizes(layer))
+    cap = per_step * args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    for e in ev_s + ev_e:
+        e.record(stream)                    # creates the underlying cudaEvent
+    arr_s = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_s])
+    arr_e = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_e])
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = lib.dq_kernel_launches()
+    lib.dq_set_timing_events(arr_s, arr_e, cap)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(mats, X)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    used = lib.dq_timing_events_used()
+    lib.dq_set_timing_events(None, None, 0)
+    launches = lib.dq_kernel_launches() - launches0
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_total = reduce_max(ms_total, world)
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    kern_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s[:used], ev_e[:used]))
+
+    ms_step = ms_total / args.steps
+    value = world * elems * T / (ms_step * 1e-3)
+
+    peaks, peak_src = _peaks()
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = 148 * 128 * sm_max * 1e6 / 1e12                         # Tops/s FP32
+    ops = args.steps * elems * (OPS_PER_ELEM_ITER * T + OPS_PER_ELEM_INIT)
+    achieved = ops / (kern_ms * 1e-3) / 1e12 if kern_ms > 0 else None
+    hbm_equiv = args.steps * elems * T * HBM_BYTES_PER_ELEM_ITER / (kern_ms * 1e-3) / 1e9
+    roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tops/s",
+            "frac": achieved / alu_peak if achieved else None, "traffic": None,
+            "peak_source": "148 SMs x 128 FP32 lanes x %.0f MHz (FMA = 1 op)" % sm_max,
+            "kernel": "solve_kernel", "kernel_ms_per_step": kern_ms / args.steps,
+            "launches_timed": used,
+            "hbm_equivalent": {"bytes_per_elem_iter": HBM_BYTES_PER_ELEM_ITER,
+                               "achieved_GBps": hbm_equiv,
+                               "frac_of_hbm_peak": hbm_equiv / float(peaks["hbm_gbs"]),
+                               "peak_GBps": float(peaks["hbm_gbs"]), "peak_source": peak_src}}
+
+    # ------------------------------------------------------------------ end to end
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elems, T)
+
+    # ------------------------------------------------------------------ CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        Wk = Ws[k0].float().cpu().numpy().astype(np.float64)
+        amax = float(np.max(np.abs(Wk)))
+        v, dt, n_el = cpu_sample_solve(Wk, amax, T)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "block-0 k_proj (1024x4096) of this layer set, 16 iterations, "
+                         "%.1f s, single process" % dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "Llama-3.1-8B-shaped layer set (%d matrices, %.3e bf16 "
+                                   "weights per GPU), NVFP4, %d BCD iterations + activation "
+                                   "rescale/NVFP4 quant 8192x4096" % (count, elems, T),
+                       "full_model_solve_s": ms_step * 1e-3,
+                       "l2": "inputs larger than L2 (%.1f GB of weights per step)"
+                             % (elems * 2 / 1e9),
+                       "parallelism": "one layer set per GPU (weak)",
+                       "blocks": args.blocks if args.blocks is not None else cfg.blocks},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def _group_sizes(layer):
+    sizes = {}
+    order = []
+    for _, _, m, n in layer:
+        if (m, n) not in sizes:
+            sizes[(m, n)] = 0
+            order.append((m, n))
+        sizes[(m, n)] += 1
+    return [sizes[k] for k in order]
+
+
+def run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elems, T):
+    """Same step through the public API from pinned host buffers, results read back."""
+    host_W = [torch.empty(W.shape, dtype=W.dtype, pin_memory=True) for W in Ws]
+    for h, W in zip(host_W, Ws):
+        h.copy_(W)
+    host_X = torch.empty(X.shape, dtype=X.dtype, pin_memory=True)
+    host_X.copy_(X)
+    dev_W = [torch.empty_like(W) for W in Ws]
+    dev_X = torch.empty_like(X)
+    mats = mats_for(dev_W)
+    keys = ("q_packed", "block_scales", "c", "tensor_scale", "mse")
+    host_out = [{k: torch.empty(o[k].shape, dtype=o[k].dtype, pin_memory=True) for k in keys}
+                for o in outs]
+    host_act = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                for k, v in act_out.items()}
+    h2d = sum(h.numel() * h.element_size() for h in host_W) + host_X.numel() * host_X.element_size()
+    d2h = sum(o[k].numel() * o[k].element_size() for o in outs for k in keys) + \
+        sum(v.numel() * v.element_size() for v in act_out.values())
+
+    def e2e_step():
+        for h, d in zip(host_W, dev_W):
+            d.copy_(h, non_blocking=True)
+        dev_X.copy_(host_X, non_blocking=True)
+        step(mats, dev_X)
+        for o, ho in zip(outs, host_out):
+            for k in keys:
+                ho[k].copy_(o[k], non_blocking=True)
+        for k, v in act_out.items():
+            host_act[k].copy_(v, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(a.elapsed_time(b), world) / args.steps
+    return {"value": world * elems * T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

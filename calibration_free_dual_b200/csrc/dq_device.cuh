@@ -1,0 +1,187 @@
+// dq_device.cuh — device-side codecs and projections shared by the DualQuant kernels.
+//
+// Element grids: INT4 (-7..7) and E2M1 (OCP MX v1.0 FP4); block scales: bf16, E8M0 and
+// E4M3 (FN) times an fp32 tensor scale. Every rounding is round-to-nearest-even on a binary32
+// input (E8M0: nearest power of two, tie up), saturating at the grid's largest magnitude.
+// Pi_S maps a scale to the nearest member of the format's set of representable block
+// scales: the projection step that the DualQuant abstract (acceptodds.com/papers/
+// iclr2027-49818) applies after every scale update.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace dq {
+
+enum Elem : int { ELEM_INT4 = 0, ELEM_E2M1 = 1 };
+enum Scale : int { SCALE_BF16 = 0, SCALE_E8M0 = 1, SCALE_E4M3 = 2 };
+
+// error bits of the per-device error word
+constexpr unsigned ERRBIT_NONFINITE = 1u;
+constexpr unsigned ERRBIT_TIMEOUT = 2u;
+constexpr unsigned ERRBIT_BADWARM = 4u;
+
+constexpr float NVFP4_TENSOR_DIV = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
+
+// ------------------------------------------------------------------ bf16 <-> fp32 (exact)
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) {
+  return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ bool bf16x2_nonfinite(uint32_t u) {
+  return ((u & 0x7F80u) == 0x7F80u) || ((u & 0x7F800000u) == 0x7F800000u);
+}
+
+// ------------------------------------------------------------------ E2M1 elements
+// Two binary32 values -> one byte of two E2M1 codes (low nibble = lo), RNE, saturating.
+__device__ __forceinline__ uint32_t e2m1x2_encode(float lo, float hi) {
+  uint16_t out;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tmov.b16 %0, {t, 0};\n\t}"
+      : "=h"(out) : "f"(lo), "f"(hi));
+  return out;
+}
+// One byte of two E2M1 codes -> their values (low nibble -> .x).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
+  uint32_t h2;
+  uint16_t b = (uint16_t)(byte & 0xFFu);
+  asm("{\n\t.reg .b8 t, tz;\n\tmov.b16 {t, tz}, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h2) : "h"(b));
+  __half2 hv = *reinterpret_cast<__half2*>(&h2);
+  return __half22float2(hv);
+}
+
+// ------------------------------------------------------------------ INT4 elements
+__device__ __forceinline__ float int4_round(float x) {
+  return fminf(fmaxf(rintf(x), -7.0f), 7.0f);
+}
+__device__ __forceinline__ uint32_t int4_code(float q) { return ((int)q) & 0xF; }
+
+// Quantize a pair on the element grid: values into q, code byte (low nibble = x.x).
+template <int ELEM>
+__device__ __forceinline__ uint32_t quant2(float2 x, float2& q) {
+  if constexpr (ELEM == ELEM_E2M1) {
+    uint32_t code = e2m1x2_encode(x.x, x.y);
+    q = e2m1x2_decode(code);
+    return code;
+  } else {
+    q.x = int4_round(x.x);
+    q.y = int4_round(x.y);
+    return int4_code(q.x) | (int4_code(q.y) << 4);
+  }
+}
+
+// ------------------------------------------------------------------ E4M3 (FN)
+// Nearest E4M3 code of u >= 0 (RNE, saturating at 448); code 0 for u that rounds to 0.
+__device__ __forceinline__ uint32_t e4m3_encode(float u) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(u));
+  return out & 0xFFu;
+}
+__device__ __forceinline__ float e4m3_decode(uint32_t code) {
+  uint32_t h2;
+  uint16_t b = (uint16_t)(code & 0xFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+  __half2 hv = *reinterpret_cast<__half2*>(&h2);
+  return __low2float(hv);
+}
+
+// ------------------------------------------------------------------ E8M0
+// Exact 2^k for k in [-149, 127].
+__device__ __forceinline__ float pow2_exact(int k) {
+  return (k >= -126) ? __uint_as_float((uint32_t)(k + 127) << 23)
+                     : __uint_as_float(1u << (k + 149));
+}
+// Code k+127 of the power of two nearest to v (tie at 1.5*2^k goes up), k in [-127, 127];
+// v <= 0 (only reachable through underflow) gives the smallest, 2^-127.
+__device__ __forceinline__ uint32_t e8m0_encode(float v) {
+  if (!(v > 0.0f)) return 0u;
+  uint32_t b = __float_as_uint(v);
+  int E = (int)(b >> 23);
+  uint32_t M = b & 0x7FFFFFu;
+  int k;
+  if (E == 0) {
+    k = (M >= 0x600000u) ? -126 : -127;   // subnormal: nearest of 2^-127, 2^-126
+  } else if (E == 255) {
+    k = 127;
+  } else {
+    k = E - 127 + (M >= 0x400000u ? 1 : 0);
+  }
+  k = max(-127, min(127, k));
+  return (uint32_t)(k + 127);
+}
+__device__ __forceinline__ float e8m0_decode(uint32_t code) { return pow2_exact((int)code - 127); }
+
+// ------------------------------------------------------------------ bf16 scale
+__device__ __forceinline__ uint32_t bf16_rn_bits(float v) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// ------------------------------------------------------------------ projection Pi_S
+struct ScaleVal {
+  float r;        // decoded scale
+  float ir;       // fl32(1 / r)
+  uint32_t code;  // stored code
+};
+
+// Decode a stored scale code. `tbl` (E4M3 only) holds fl32(s_t*e) and fl32(1/that) per code.
+template <int SCALE>
+__device__ __forceinline__ ScaleVal scale_decode(uint32_t code, const float2* tbl) {
+  ScaleVal s;
+  s.code = code;
+  if constexpr (SCALE == SCALE_BF16) {
+    s.r = __uint_as_float(code << 16);
+    s.ir = __frcp_rn(s.r);
+  } else if constexpr (SCALE == SCALE_E8M0) {
+    s.r = pow2_exact((int)code - 127);
+    s.ir = pow2_exact(127 - (int)code);
+  } else {
+    float2 t = tbl[code];
+    s.r = t.x;
+    s.ir = t.y;
+  }
+  return s;
+}
+
+// Nearest admissible scale to v (binary32): bf16 RNE clamped to [2^-126, max]; E8M0 nearest
+// power of two; E4M3: e = RNE(fl32(v / s_t)) raised to 2^-9 if 0, scale fl32(s_t * e).
+template <int SCALE>
+__device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const float2* tbl) {
+  uint32_t code;
+  if constexpr (SCALE == SCALE_BF16) {
+    code = (v > 0.0f) ? bf16_rn_bits(v) : 0x0080u;
+    code = min(max(code, 0x0080u), 0x7F7Fu);
+  } else if constexpr (SCALE == SCALE_E8M0) {
+    code = e8m0_encode(v);
+  } else {
+    float u = (v > 0.0f) ? __fdiv_rn(v, s_t) : 0.0f;
+    code = max(e4m3_encode(u), 1u);
+  }
+  return scale_decode<SCALE>(code, tbl);
+}
+
+// Same projection without the per-CTA E4M3 table (decoded scale computed directly).
+template <int SCALE>
+__device__ __forceinline__ ScaleVal project_scale_direct(float v, float s_t) {
+  if constexpr (SCALE == SCALE_E4M3) {
+    const float u = (v > 0.0f) ? __fdiv_rn(v, s_t) : 0.0f;
+    ScaleVal sv;
+    sv.code = max(e4m3_encode(u), 1u);
+    sv.r = __fmul_rn(s_t, e4m3_decode(sv.code));
+    sv.ir = __frcp_rn(sv.r);
+    return sv;
+  } else {
+    return project_scale<SCALE>(v, s_t, nullptr);
+  }
+}
+
+// NVFP4 per-tensor scale from the amax bit pattern.
+__device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
+  return (amax > 0.0f) ? __fdiv_rn(amax, NVFP4_TENSOR_DIV) : 1.0f;
+}
+
+// ------------------------------------------------------------------ packed fp32x2 math
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+}  // namespace dq

@@ -1,0 +1,108 @@
+// dq_internal.h — launch descriptors shared by the host API and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dq {
+
+constexpr int SOLVE_NT = 256;          // threads per CTA of the solve kernel
+constexpr int SOLVE_MAXMATS = 32;      // matrices per solve launch (descriptors by value)
+constexpr int SOLVE_MAXK = 8;          // CTAs per cluster (portable cluster size)
+constexpr size_t SOLVE_WTILE_MAX = 96 * 1024;   // bytes of W kept per CTA
+
+struct SolveMat {
+  const void* W;
+  int64_t ldw;
+  const float* r0;
+  const float* c0;
+  uint8_t* q_packed;
+  float* r;
+  float* c;
+  void* bscale;
+  float* tensor_scale;
+  double* ws_err;              // [(T+1) * tiles] per-iteration partial errors
+  double* ws_wsq;              // [tiles] partial ||W||^2
+  unsigned* amax_bits;         // NVFP4: amax |W| as float bits (zeroed before the pre-pass)
+};
+
+struct SolveLaunch {
+  int m, n, T, K, R, tiles;
+  unsigned* err_word;
+  SolveMat mats[SOLVE_MAXMATS];
+};
+
+struct SolvePlan {
+  int S;        // 16-column segments per CTA tile (tile width TN = 16*S)
+  int K;        // CTAs per cluster (row split of one column strip)
+  int R;        // rows per CTA
+  int tiles;    // column tiles per matrix (n / TN)
+  size_t smem;  // dynamic shared memory per CTA
+};
+
+// Shared-memory carve-up of a solve CTA (same arithmetic on host and device).
+struct SolveSmem {
+  size_t w, codes, tbl, cvec, icvec, red, slot, colsum, errv, total;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize, int scb) {
+  const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
+  SolveSmem l;
+  size_t off = 0;
+  l.w = off;      off = align_up(off + (size_t)R * TN * esize, 128);
+  l.codes = off;  off = align_up(off + (size_t)R * NBLK * scb, 16);
+  l.tbl = off;    off = align_up(off + 128 * 8, 16);
+  l.cvec = off;   off = align_up(off + TN * 4, 16);
+  l.icvec = off;  off = align_up(off + TN * 4, 16);
+  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * 32 * 4, 16);
+  l.slot = off;   off = align_up(off + (size_t)2 * 64 * S * 8, 16);
+  l.colsum = off; off = align_up(off + TN * 8, 16);
+  l.errv = off;   off = align_up(off + TN * 8, 16);
+  l.total = off;
+  return l;
+}
+
+// format helpers (kind as in dq.h)
+inline int fmt_block(int kind, int group) {
+  switch (kind) {
+    case 0: return (group == 64 || group == 128) ? group : 0;
+    case 1: case 2: return group == 32 ? 32 : 0;
+    case 3: return group == 16 ? 16 : 0;
+    default: return 0;
+  }
+}
+
+// measurement hooks (dq_api.cu)
+void count_launches(int n);
+void timing_before(cudaStream_t s);
+void timing_after(cudaStream_t s);
+
+bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ctas_hint,
+                SolvePlan* p);
+cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
+                         const SolvePlan& p, cudaStream_t s);
+cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s);
+cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* const* ws_wsq,
+                            const int* tiles, int count, int T, cudaStream_t s);
+
+struct ActLaunch {
+  const void* X;
+  int64_t tokens, n, ldx;
+  const float* c;
+  uint8_t* x_packed;
+  void* scales;
+  float* tensor_scale;
+  unsigned* amax_bits;
+  unsigned* err_word;
+};
+cudaError_t launch_act(const ActLaunch& A, int kind, int group, int esize, cudaStream_t s);
+
+cudaError_t launch_encode(const float* x, int64_t count, int codec, void* codes,
+                          cudaStream_t s);
+cudaError_t launch_decode(const void* codes, int64_t count, int codec, float* x,
+                          cudaStream_t s);
+
+}  // namespace dq

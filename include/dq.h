@@ -1,0 +1,177 @@
+/*
+ * dq.h — C ABI of the DualQuant dual-scale solver for NVIDIA B200 (sm_100a).
+ *
+ * What is computed is the DualQuant hot path ("DualQuant: Dual-scale Calibration-free
+ * Weight-and-Activation Quantization for LLMs"): for each weight matrix W (m x n,
+ * out_features x in_features) a row-block scale r, a column scale c and 4-bit codes Q with
+ * W ~ diag(r) Q diag(c), fitted by block coordinate descent with closed-form updates
+ * (Abstract), the quantizer used as a black box and the scales projected onto the
+ * format's admissible set after every update (acceptodds.com abstract of the same paper);
+ * and the activation rescale by the column scales followed by 4-bit quantization
+ * (Abstract; appendix Table 11, "Activation quantization (incl. beta)").
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are CUDA device pointers; "host" are host pointers.
+ *  - The caller allocates every buffer, including the workspace; the library never
+ *    allocates, frees or keeps a pointer after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream). Outputs are valid once the stream has been synchronised.
+ *  - Argument errors are returned synchronously before any work is queued. Conditions
+ *    found on the device (non-finite input) raise a per-device error word that
+ *    dq_last_device_error() reads and clears.
+ *  - Layouts are row-major. Element codes are packed two per byte, the low nibble holding
+ *    the even column. Block scales are stored one code per block: INT4 -> uint16 bf16 bit
+ *    pattern, MXINT4/MXFP4 -> uint8 E8M0 (2^(code-127)), NVFP4 -> uint8 E4M3 multiplied by
+ *    the fp32 tensor scale.
+ */
+#ifndef DQ_H_
+#define DQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DQ_API __attribute__((visibility("default")))
+#else
+#define DQ_API
+#endif
+
+typedef enum {
+  DQ_OK = 0,
+  DQ_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad stride or alignment      */
+  DQ_ERR_SHAPE = 2,         /* n not a multiple of the format's block length, too large  */
+  DQ_ERR_DTYPE = 3,         /* unknown dtype / format / codec                            */
+  DQ_ERR_WORKSPACE = 4,     /* workspace smaller than the *_workspace_bytes() figure     */
+  DQ_ERR_NONFINITE = 5,     /* a NaN or Inf was found in an input (device-detected)      */
+  DQ_ERR_TIMEOUT = 6,       /* a bounded device wait gave up (device-detected)           */
+  DQ_ERR_CUDA = 7,          /* a CUDA runtime call failed                                */
+  DQ_ERR_UNSUPPORTED = 8    /* a shape the kernels do not handle (e.g. rows too many)    */
+} dq_status;
+
+typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_MXFP4 = 2, DQ_NVFP4 = 3 } dq_kind;
+
+/* Format: kind plus block length along a row. INT4: group 64 or 128 (bf16 block scale,
+ * elements -7..7). MXINT4: 32 (E8M0, elements -7..7). MXFP4: 32 (E8M0, E2M1 elements).
+ * NVFP4: 16 (E4M3 block scale times an fp32 tensor scale, E2M1 elements). */
+typedef struct {
+  int32_t kind;
+  int32_t group;
+} dq_format;
+
+typedef enum { DQ_F32 = 0, DQ_BF16 = 1 } dq_dtype;
+
+/* One matrix of a solve. All pointers are device pointers.
+ *   W            [m, ldw] input weights (dtype of the call), 16-byte aligned, ldw*esize % 16 == 0
+ *   r0           optional warm-start row-block scales [m, n/B] fp32 (projected on entry), or NULL
+ *   c0           optional warm-start column scales [n] fp32 (finite, > 0), or NULL
+ *   q_packed     out [m, n/2] uint8, the codes of the returned state
+ *   r            out [m, n/B] fp32, decoded row-block scales
+ *   c            out [n] fp32, column scales
+ *   block_scales out [m, n/B] codes of r (uint16 for INT4, uint8 otherwise)
+ *   tensor_scale out [1] fp32, NVFP4 only (may be NULL for the other formats)
+ *   mse_trace    out [iters+1] fp64, ||W - W_hat||^2/||W||^2 after init and each iteration */
+typedef struct {
+  const void* W;
+  int64_t m, n, ldw;
+  const float* r0;
+  const float* c0;
+  uint8_t* q_packed;
+  float* r;
+  float* c;
+  void* block_scales;
+  float* tensor_scale;
+  double* mse_trace;
+} dq_matrix;
+
+/* Workspace (device bytes) needed by dq_solve_batched for these shapes. `m`, `n` are host
+ * arrays of `count` entries. Returns 0 for invalid arguments. */
+DQ_API size_t dq_solve_workspace_bytes(int64_t count, const int64_t* m, const int64_t* n,
+                                       dq_format fmt, int32_t iters);
+
+/* Dual-scale BCD solve of `count` independent matrices (a full layer set in one call).
+ * `mats` is a host array of descriptors. Per matrix: iteration 0 sets c = 1 (or c0) and
+ * r = Pi_S(absmax/q_max) (or Pi_S(r0)); then `iters` iterations of
+ *   Q-step  q = RNE_E(fl32(fl32(W * fl32(1/c)) * fl32(1/r)))
+ *   r-step  r = Pi_S(sum_b W q c / sum_b (q c)^2)     per (row, block)
+ *   c-step  c = sum_i W q r / sum_i (q r)^2           per column
+ * (DualQuant Abstract: BCD with closed-form updates; acceptodds abstract: projection of the
+ * scales after each update; Figure 2 (b): the trace, monotone by Theorem 1 (i)).
+ * Returns DQ_ERR_SHAPE if some n is not a multiple of fmt.group, DQ_ERR_UNSUPPORTED if a
+ * matrix has more rows than the cluster-resident kernel holds (see dq_solve_max_rows). */
+DQ_API dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype,
+                                  dq_format fmt, int32_t iters, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Single-matrix form of dq_solve_batched (same semantics, flat arguments). */
+DQ_API dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, int64_t ldw,
+                          dq_format fmt, int32_t iters, const float* r0, const float* c0,
+                          uint8_t* q_packed, float* r, float* c, void* block_scales,
+                          float* tensor_scale, double* mse_trace, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* Largest m the solver handles for a given n, format and dtype (0 if the format is bad). */
+DQ_API int64_t dq_solve_max_rows(int64_t n, dq_format fmt, int32_t dtype);
+
+/* Workspace (device bytes) needed by dq_act_quant. */
+DQ_API size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt);
+
+/* Activation rescale + 4-bit quantization (DualQuant Abstract: the column scales are
+ * per-channel activation rescalings applied before activation quantization; appendix
+ * Table 6: activation SQNR with and without them). With W_hat = diag(r) Q diag(c), the
+ * quantized GEMM consumes c * x, so x~ = fl32(X * c) per channel (c NULL: x~ = X). Per
+ * (token, block of B channels): a = max|x~|, d = Pi_S(a / q_max) (0 for a = 0; NVFP4 with
+ * s_t = amax(x~)/2688), q = RNE_E(fl32(x~ * fl32(1/d))).
+ *   X            device [tokens, ldx] (dtype), 16-byte aligned, ldx*esize % 16 == 0
+ *   c            device [n] fp32 or NULL
+ *   x_packed     device out [tokens, n/2] uint8
+ *   scales       device out [tokens, n/B] (uint16 bf16 bits for INT4, uint8 otherwise)
+ *   tensor_scale device out [1] fp32 (NVFP4; may be NULL otherwise) */
+DQ_API dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n,
+                              int64_t ldx, const float* c, dq_format fmt, uint8_t* x_packed,
+                              void* scales, float* tensor_scale, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Codecs used by the kernels, exposed for bit-exact tests (one code per output element). */
+typedef enum {
+  DQ_CODEC_INT4 = 0,   /* RNE to -7..7, saturating; code = two's-complement nibble (uint8) */
+  DQ_CODEC_E2M1 = 1,   /* RNE to E2M1, saturating at 6; code = sign<<3 | magnitude (uint8) */
+  DQ_CODEC_E4M3 = 2,   /* RNE to E4M3 (FN), saturating at 448 (uint8)                      */
+  DQ_CODEC_E8M0 = 3,   /* nearest power of two, tie up, clamped to 2^-127..2^127 (uint8)  */
+  DQ_CODEC_BF16 = 4    /* RNE to bfloat16 (uint16 bit pattern)                             */
+} dq_codec;
+
+/* x: device fp32 [count]; codes: device [count] of the codec's code type. */
+DQ_API dq_status dq_encode(const float* x, int64_t count, int32_t codec, void* codes,
+                           void* stream);
+/* codes: device [count]; x: device fp32 [count] decoded values. */
+DQ_API dq_status dq_decode(const void* codes, int64_t count, int32_t codec, float* x,
+                           void* stream);
+
+/* Synchronises `stream`, then returns and clears the device error word of the current
+ * device: DQ_ERR_NONFINITE, DQ_ERR_TIMEOUT or DQ_OK (DQ_ERR_CUDA if a CUDA call fails). */
+DQ_API dq_status dq_last_device_error(void* stream);
+
+/* Measurement hooks (no computation). dq_set_timing_events: before the i-th launch of the
+ * solve kernel made by this host thread the library records start_events[i] on the launch
+ * stream and after it stop_events[i], for i < capacity; the events (cudaEvent_t, created by
+ * the caller with timing enabled) stay the caller's. NULL / 0 disables. Returns
+ * DQ_ERR_INVALID_ARG for a negative capacity or a NULL array with capacity > 0. */
+DQ_API dq_status dq_set_timing_events(void* const* start_events, void* const* stop_events,
+                                      int32_t capacity);
+/* Number of solve-kernel launches recorded since the last dq_set_timing_events call. */
+DQ_API int32_t dq_timing_events_used(void);
+/* Kernels this library has launched from this process so far (all entry points). */
+DQ_API int64_t dq_kernel_launches(void);
+
+/* Human-readable name of a status code (static storage). */
+DQ_API const char* dq_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_H_ */

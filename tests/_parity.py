@@ -1,0 +1,113 @@
+"""Comparison of CUDA-path outputs with the oracle (test helper, not collected).
+
+Tolerances (the solver's floating-point tolerance, written out here once):
+  * element codes: >= 99.9% identical; every mismatch is one grid step away and sits either
+    in a block whose scale differs between the two sides or next to a rounding midpoint;
+  * block scales (discrete, on the admissible set): >= 99.9% identical, mismatches one
+    admissible step apart;
+  * column scales c: ||c_gpu - c_ora||_2 / ||c_ora||_2 <= 1e-4;
+  * normalised MSE trace: |mse_gpu - mse_ora| / mse_ora <= 1e-4 at every iteration;
+  * NVFP4 tensor scale: bit-exact.
+Identical binary32 state gives identical codes (the decision is taken on the same binary32
+quotient); the residual differences come from summation order (binary32 block sums on the
+GPU vs binary64 in the oracle), which can move a projection or a code across a midpoint.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import formats as F
+
+CODE_MATCH = 0.999
+SCALE_MATCH = 0.999
+C_REL = 1e-4
+MSE_REL = 1e-4
+
+
+def oracle_format(name_or_spec):
+    if isinstance(name_or_spec, str):
+        kind, group = {"INT4": ("INT4", 128), "INT4_G64": ("INT4", 64),
+                       "MXINT4": ("MXINT4", 32), "MXFP4": ("MXFP4", 32),
+                       "NVFP4": ("NVFP4", 16)}[name_or_spec]
+    else:
+        kind, group = name_or_spec.kind, name_or_spec.group
+    return F.make_format(kind, group)
+
+
+def to_host(out: dict) -> dict:
+    h = {}
+    for k, v in out.items():
+        if k.startswith("_"):
+            continue
+        h[k] = v.detach().cpu().numpy()
+    return h
+
+
+def grid_index(q: np.ndarray, fmt) -> np.ndarray:
+    """Position of each element value on the signed grid (-0 and +0 coincide)."""
+    if fmt.elem == "int4":
+        return np.rint(q).astype(np.int64)
+    mag = np.abs(q)
+    idx = np.searchsorted(F.E2M1_MAG, mag)
+    return np.where(q < 0, -idx, idx)
+
+
+def scale_codes_gpu(h: dict, fmt) -> np.ndarray:
+    bs = h["block_scales"]
+    if fmt.scale == "bf16":
+        return bs.view(np.uint16).astype(np.int64)
+    return bs.astype(np.int64)
+
+
+def scale_step(code_a: np.ndarray, code_b: np.ndarray, fmt) -> np.ndarray:
+    """Distance in admissible steps between two scale codes."""
+    return np.abs(code_a.astype(np.int64) - code_b.astype(np.int64))
+
+
+def compare_solve(h: dict, ora: dict, fmt, *, exact: bool = False, label: str = "") -> dict:
+    """Assert the parity bar; return the measured agreement figures."""
+    codes_g = F.unpack_codes(h["q_packed"])
+    codes_o = ora["codes"]
+    qg = F.decode_elem(codes_g, fmt)
+    qo = ora["q"]
+    same_q = (grid_index(qg, fmt) == grid_index(qo, fmt))
+    sc_g = scale_codes_gpu(h, fmt)
+    sc_o = np.asarray(ora["r_codes"]).astype(np.int64)
+    same_r = sc_g == sc_o
+    rep = dict(code_match=float(same_q.mean()), scale_match=float(same_r.mean()))
+    rep["c_rel"] = float(np.linalg.norm(h["c"].astype(np.float64) - ora["c"]) /
+                         max(np.linalg.norm(ora["c"].astype(np.float64)), 1e-300))
+    mo = np.asarray(ora["mse"])
+    mg = h["mse"]
+    rel = np.abs(mg - mo) / np.maximum(np.abs(mo), 1e-300)
+    rel = np.where(mo == 0, np.abs(mg - mo), rel)
+    rep["mse_rel_max"] = float(rel.max())
+    if exact:
+        assert same_q.all(), (label, "codes differ", int((~same_q).sum()))
+        assert same_r.all(), (label, "scales differ", int((~same_r).sum()))
+    assert rep["code_match"] >= CODE_MATCH, (label, rep)
+    assert rep["scale_match"] >= SCALE_MATCH, (label, rep)
+    # mismatched codes: one grid step, or their block scale differs
+    B = fmt.block
+    blk_diff = np.repeat(~same_r, B, axis=1)
+    step = np.abs(grid_index(qg, fmt) - grid_index(qo, fmt))
+    bad = (~same_q) & (step > 1) & (~blk_diff)
+    assert not bad.any(), (label, "code mismatches beyond one step", int(bad.sum()))
+    # mismatched scales: one admissible step
+    if fmt.scale == "bf16":
+        st = scale_step(sc_g, sc_o, fmt)
+    else:
+        st = scale_step(sc_g, sc_o, fmt)
+    assert np.all(st[~same_r] <= 1), (label, "scale mismatches beyond one step")
+    # decoded r consistent with the codes (exactly)
+    rg = h["r"]
+    if fmt.scale != "e4m3":
+        np.testing.assert_array_equal(rg, F.decode_scale(sc_g, fmt))
+    assert rep["c_rel"] <= C_REL, (label, rep)
+    assert rep["mse_rel_max"] <= MSE_REL, (label, rep)
+    return rep
+
+
+def assert_monotone(mse: np.ndarray, rel: float = 1e-6, label: str = "") -> None:
+    assert np.all(mse[1:] <= mse[:-1] * (1 + rel)), (label, mse)

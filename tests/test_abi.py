@@ -1,0 +1,103 @@
+"""The C ABI library loads and exports what include/dq.h declares; host-side validation
+rejects bad arguments before any CUDA call (CPU only, no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dq():
+    from calibration_free_dual_b200 import build
+    build.build()
+    import calibration_free_dual_b200 as pkg
+    return pkg
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"DQ_API\s+[\w\s\*]+?\b(dq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for must in ["dq_solve", "dq_solve_batched", "dq_solve_workspace_bytes", "dq_act_quant",
+                 "dq_act_quant_workspace_bytes", "dq_encode", "dq_decode",
+                 "dq_last_device_error", "dq_status_string", "dq_solve_max_rows"]:
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(dq):
+    lib = ctypes.CDLL(dq._lib.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    # and nothing else with the dq_ prefix is missing from the binding
+    for name in _declared():
+        assert name in dq._lib.SIGNATURES, name
+
+
+def test_exports_are_only_the_c_abi(dq):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", dq._lib.LIB_PATH],
+                         stdout=subprocess.PIPE, text=True).stdout
+    text_syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert sorted(text_syms) == _declared()
+
+
+def test_status_strings(dq):
+    assert dq.dq_status_string(0) == b"DQ_OK"
+    assert dq.dq_status_string(2) == b"DQ_ERR_SHAPE"
+    assert dq.dq_status_string(99) == b"DQ_ERR_UNKNOWN"
+
+
+def test_validation_happens_before_cuda(dq):
+    f = dq.fmt_of("NVFP4")
+    nul = None
+    # n not a multiple of the block length
+    assert dq.dq_solve(nul, 1, 64, 100, 100, f, 4, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 2
+    # null W with a valid shape
+    assert dq.dq_solve(nul, 1, 64, 128, 128, f, 4, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 1
+    # bad format / dtype
+    bad = dq.dq_format(3, 32)
+    assert dq.dq_solve(nul, 1, 64, 128, 128, bad, 4, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 3
+    assert dq.dq_solve(nul, 7, 64, 128, 128, f, 4, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 3
+    # negative iterations, ldw < n
+    assert dq.dq_solve(nul, 1, 64, 128, 128, f, -1, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 1
+    assert dq.dq_solve(nul, 1, 64, 128, 64, f, 4, nul, nul, nul, nul, nul, nul, nul, nul,
+                       nul, 0, nul) == 1
+    # act quant shape / workspace checks
+    assert dq.dq_act_quant(nul, 1, 8, 100, 100, nul, f, nul, nul, nul, nul, 0, nul) == 2
+    assert dq.dq_act_quant(nul, 1, 8, 128, 128, nul, f, nul, nul, nul, nul, 0, nul) == 1
+    assert dq.dq_encode(nul, 4, 9, nul, nul) == 3
+    assert dq.dq_decode(nul, -1, 1, nul, nul) == 1
+
+
+def test_workspace_bytes_and_limits(dq):
+    f = dq.fmt_of("NVFP4")
+    m = (ctypes.c_int64 * 2)(4096, 14336)
+    n = (ctypes.c_int64 * 2)(4096, 4096)
+    one = dq.dq_solve_workspace_bytes(1, m, n, f, 16)
+    two = dq.dq_solve_workspace_bytes(2, m, n, f, 16)
+    assert 0 < one < two
+    assert dq.dq_solve_workspace_bytes(1, m, (ctypes.c_int64 * 1)(100), f, 16) == 0
+    assert dq.dq_solve_max_rows(4096, f, 1) >= 14336            # 8B-shaped gate/up fit
+    assert dq.dq_solve_max_rows(4096, dq.fmt_of("MXFP4"), 1) >= 11008
+    assert dq.dq_solve_max_rows(512, dq.fmt_of("INT4"), 0) >= 512
+    assert dq.dq_act_quant_workspace_bytes(8192, 4096, f) > 0
+
+
+def test_no_cpu_fallback(dq):
+    import torch
+    with pytest.raises(TypeError):
+        dq.solve(torch.zeros(16, 32), "NVFP4", 2)
+    with pytest.raises(TypeError):
+        dq.act_quant(torch.zeros(4, 32), "NVFP4")

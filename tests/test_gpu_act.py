@@ -1,0 +1,99 @@
+"""Parity of the CUDA activation rescale + 4-bit quantization with the oracle (B200).
+
+Every decision in this path is taken on the same binary32 values on both sides (the
+product X*c, the block maximum, fl32(a/q_max), the scale projection and fl32(x*1/d)), so
+codes and scale codes must agree bit for bit, and the SQNRs computed from them agree.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import formats as F
+from oracle import solver as S
+from oracle.actquant import act_quant as ora_act, dequant, sqnr
+from tests._parity import oracle_format
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dq():
+    import calibration_free_dual_b200 as pkg
+    return pkg
+
+
+def _gpu_act(dq, X, fmt_name, c):
+    o = dq.act_quant(X.cuda(), fmt_name, None if c is None else torch.from_numpy(c).cuda())
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    return {k: v.cpu().numpy() for k, v in o.items() if not k.startswith("_")}
+
+
+def _check(h, ora, fmt):
+    codes = F.unpack_codes(h["x_packed"])
+    np.testing.assert_array_equal(codes, ora["codes"])
+    sc = h["scales"].view(np.uint16) if fmt.scale == "bf16" else h["scales"]
+    np.testing.assert_array_equal(sc.astype(np.int64), ora["scale_codes"].astype(np.int64))
+    if fmt.kind == "NVFP4":
+        assert np.float32(h["tensor_scale"][0]) == ora["s_t"]
+
+
+def _decode_gpu(h, fmt):
+    codes = F.unpack_codes(h["x_packed"])
+    q = F.decode_elem(codes, fmt)
+    sc = h["scales"].view(np.uint16) if fmt.scale == "bf16" else h["scales"]
+    s_t = h["tensor_scale"][0] if fmt.kind == "NVFP4" else None
+    d = F.decode_scale(sc, fmt, s_t).astype(np.float64)
+    if fmt.scale == "bf16":
+        d = np.where(sc == 0, 0.0, d)
+    return dequant(d, q, fmt.block)
+
+
+@pytest.mark.parametrize("fmt_name", ["NVFP4", "INT4", "INT4_G64", "MXFP4", "MXINT4"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_act_quant_bit_exact(dq, fmt_name, dtype):
+    rng = np.random.default_rng(3)
+    T, n = 77, 1280                       # ragged last 256-channel round, odd token count
+    X = rng.standard_normal((T, n)).astype(np.float32)
+    X[:, rng.choice(n, 4, replace=False)] *= 50
+    X[5, :] = 0.0                          # an all-zero token row
+    c = rng.uniform(0.25, 3.0, n).astype(np.float32)
+    Xt = torch.from_numpy(X)
+    if dtype == "bf16":
+        Xt = Xt.to(torch.bfloat16)
+    fmt = oracle_format(fmt_name)
+    Xn = Xt.float().numpy()
+    for cc in (c, None):
+        h = _gpu_act(dq, Xt, fmt_name, cc)
+        ora = ora_act(Xn, fmt, cc)
+        _check(h, ora, fmt)
+
+
+def test_act_quant_config_sqnr(dq):
+    """8192 tokens x 4096 channels with six x50 channels; c from the oracle's MXFP4 solve of
+    a 1024x4096 k_proj drawn with the Student-t recipe. SQNR with and without c agree."""
+    cfg = wl.ACT_KPROJ
+    Wk = wl.weight_host(cfg, 0, 1)
+    c = S.solve(Wk.float().numpy().astype(np.float64), oracle_format("MXFP4"), cfg.iters)["c"]
+    X = wl.act_host()
+    Xn = X.float().numpy()
+    for fmt_name in ("NVFP4", "INT4"):
+        fmt = oracle_format(fmt_name)
+        res = {}
+        for tag, cc in (("with_c", c), ("without_c", None)):
+            h = _gpu_act(dq, X, fmt_name, cc)
+            ora = ora_act(Xn, fmt, cc)
+            _check(h, ora, fmt)
+            s_gpu = sqnr(ora["xt"], _decode_gpu(h, fmt))
+            s_ora = sqnr(ora["xt"], dequant(ora["d"], ora["q"], fmt.block))
+            assert abs(s_gpu - s_ora) <= 1e-4
+            res[tag] = s_gpu
+        assert all(np.isfinite(v) and v > 5 for v in res.values()), res
+
+
+def test_act_nonfinite_reported(dq):
+    X = torch.randn(8, 64)
+    X[2, 3] = float("inf")
+    dq.act_quant(X.cuda(), "MXFP4")
+    assert dq.last_device_error() == 5
