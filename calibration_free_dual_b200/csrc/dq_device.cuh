@@ -160,6 +160,26 @@ __device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const floa
   return scale_decode<SCALE>(code, tbl);
 }
 
+// Projection of the least-squares scale num/den inside a BCD iteration. The quotient is a
+// binary32 approximation (its summands are binary32 sums already): fast division, and for
+// E4M3 the scaled quotient num / (den * s_t) directly.
+template <int SCALE>
+__device__ __forceinline__ ScaleVal project_scale_ls(float num, float den, float s_t,
+                                                     const float2* tbl) {
+  uint32_t code;
+  if constexpr (SCALE == SCALE_BF16) {
+    const float v = __fdividef(num, den);
+    code = (v > 0.0f) ? bf16_rn_bits(v) : 0x0080u;
+    code = min(max(code, 0x0080u), 0x7F7Fu);
+  } else if constexpr (SCALE == SCALE_E8M0) {
+    code = e8m0_encode(__fdividef(num, den));
+  } else {
+    const float u = __fdividef(num, __fmul_rn(den, s_t));
+    code = max(e4m3_encode(u > 0.0f ? u : 0.0f), 1u);
+  }
+  return scale_decode<SCALE>(code, tbl);
+}
+
 // Same projection without the per-CTA E4M3 table (decoded scale computed directly).
 template <int SCALE>
 __device__ __forceinline__ ScaleVal project_scale_direct(float v, float s_t) {

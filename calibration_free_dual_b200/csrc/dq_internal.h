@@ -10,7 +10,8 @@ namespace dq {
 constexpr int SOLVE_NT = 256;          // threads per CTA of the solve kernel
 constexpr int SOLVE_MAXMATS = 32;      // matrices per solve launch (descriptors by value)
 constexpr int SOLVE_MAXK = 8;          // CTAs per cluster (portable cluster size)
-constexpr size_t SOLVE_WTILE_MAX = 96 * 1024;   // bytes of W kept per CTA
+constexpr size_t SOLVE_WTILE_MAX = 64 * 1024;    // preferred: 3 CTAs per SM
+constexpr size_t SOLVE_WTILE_BIG = 200 * 1024;   // ceiling for tall strips   // bytes of W kept per CTA
 
 struct SolveMat {
   const void* W;
@@ -34,7 +35,7 @@ struct SolveLaunch {
 };
 
 struct SolvePlan {
-  int S;        // 16-column segments per CTA tile (tile width TN = 16*S)
+  int S;        // 8-column segments per CTA tile (tile width TN = 8*S)
   int K;        // CTAs per cluster (row split of one column strip)
   int R;        // rows per CTA
   int tiles;    // column tiles per matrix (n / TN)
@@ -49,7 +50,7 @@ struct SolveSmem {
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize, int scb) {
-  const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
+  const int TN = 8 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
   SolveSmem l;
   size_t off = 0;
   l.w = off;      off = align_up(off + (size_t)R * TN * esize, 128);
@@ -57,10 +58,10 @@ __host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize
   l.tbl = off;    off = align_up(off + 128 * 8, 16);
   l.cvec = off;   off = align_up(off + TN * 4, 16);
   l.icvec = off;  off = align_up(off + TN * 4, 16);
-  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * 32 * 4, 16);
-  l.slot = off;   off = align_up(off + (size_t)2 * 64 * S * 8, 16);
+  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * 16 * 4, 16);
+  l.slot = off;   off = align_up(off + (size_t)2 * 32 * S * 8, 16);
   l.colsum = off; off = align_up(off + TN * 8, 16);
-  l.errv = off;   off = align_up(off + TN * 8, 16);
+  l.errv = off;
   l.total = off;
   return l;
 }

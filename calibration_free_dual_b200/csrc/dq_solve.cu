@@ -22,6 +22,8 @@
 //   * one cluster barrier per iteration (double-buffered partial slots), no spin-waits.
 #include <cooperative_groups.h>
 
+#include <type_traits>
+
 #include "dq_device.cuh"
 #include "dq_internal.h"
 
@@ -31,35 +33,33 @@ namespace dq {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
+constexpr int SEG = 8;                 // columns per thread segment
 
-// 16-byte chunk position of chunk h of the 16-column piece P (row-major [R][TN] tile),
-// swizzled so that the 8 lanes of a quarter warp reading 8 consecutive pieces hit 8
-// distinct bank groups.
+// 16-byte chunk position of chunk h of the 8-column piece P (row-major [R][TN] tile).
+// bf16: one chunk per piece, 8 lanes of a quarter warp read 128 contiguous bytes.
+// fp32: two chunks per piece, swizzled so a quarter warp hits 8 distinct bank groups.
 template <int ESZ>
 __device__ __forceinline__ int chunk_pos(int P, int h) {
   if constexpr (ESZ == 2) {
-    return 2 * P + (h ^ ((P >> 2) & 1));
+    return P;
   } else {
-    return 4 * P + (h ^ ((P >> 1) & 3));
+    return 2 * P + (h ^ ((P >> 2) & 1));
   }
 }
 
 template <int ESZ>
-__device__ __forceinline__ void load_piece(const unsigned char* Wsm, int P, float2 (&w)[8]) {
+__device__ __forceinline__ void load_piece(const unsigned char* Wsm, int P, float2 (&w)[4]) {
   const uint4* base = reinterpret_cast<const uint4*>(Wsm);
   if constexpr (ESZ == 2) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint4 v = base[chunk_pos<2>(P, h)];
-      w[4 * h + 0] = bf16x2_to_f2(v.x);
-      w[4 * h + 1] = bf16x2_to_f2(v.y);
-      w[4 * h + 2] = bf16x2_to_f2(v.z);
-      w[4 * h + 3] = bf16x2_to_f2(v.w);
-    }
+    const uint4 v = base[chunk_pos<2>(P, 0)];
+    w[0] = bf16x2_to_f2(v.x);
+    w[1] = bf16x2_to_f2(v.y);
+    w[2] = bf16x2_to_f2(v.z);
+    w[3] = bf16x2_to_f2(v.w);
   } else {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      uint4 v = base[chunk_pos<4>(P, h)];
+    for (int h = 0; h < 2; ++h) {
+      const uint4 v = base[chunk_pos<4>(P, h)];
       w[2 * h + 0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
       w[2 * h + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
     }
@@ -73,20 +73,20 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// Lane L ends with values [L - s, L - s + S) of its segment's 32-vector summed over the
-// 32/S lanes that share segment s = L % S (fixed butterfly order: deterministic).
+// Butterfly reduction of a 16-value vector over the 32/S lanes sharing segment s = lane % S.
+// Lane L ends with S/2 consecutive values starting at index (L - s) / 2 (fixed order).
 template <int S>
-__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
-  int cnt = 32;
+__device__ __forceinline__ void transpose_reduce(float (&v)[16], int lane) {
+  int cnt = 16;
 #pragma unroll
   for (int off = 16; off >= S; off >>= 1) {
     const int half = cnt >> 1;
     const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < 8; ++i) {
       if (i < half) {
-        float send = upper ? v[i] : v[i + half];
-        float keep = upper ? v[i + half] : v[i];
+        const float send = upper ? v[i] : v[i + half];
+        const float keep = upper ? v[i + half] : v[i];
         v[i] = keep + __shfl_xor_sync(FULL, send, off);
       }
     }
@@ -95,13 +95,16 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
 }
 
 template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-__global__ void __launch_bounds__(SOLVE_NT, 2) solve_kernel(const __grid_constant__ SolveLaunch L) {
-  constexpr int NT = SOLVE_NT, NWARP = NT / 32, TN = 16 * S, NBLK = S / LPB, B = 16 * LPB;
-  constexpr int NG = NT / S;
+__global__ void __launch_bounds__(SOLVE_NT, (SCALE == SCALE_BF16) ? 2 : 3)
+solve_kernel(const __grid_constant__ SolveLaunch L) {
+  constexpr int NT = SOLVE_NT, NWARP = NT / 32, TN = SEG * S, NBLK = S / LPB, B = SEG * LPB;
+  constexpr int NG = NT / S;            // rows covered by one pass of all threads
+  constexpr int VPL = S / 2;            // reduced values per lane
   constexpr int ESZ = F32IN ? 4 : 2;
+  constexpr int CPP = ESZ / 2;          // 16-byte chunks per 8-column piece
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
   constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
-  static_assert(NBLK * LPB == S, "tile must hold whole blocks");
+  static_assert(NBLK * LPB == S && S >= 2 && S <= 16, "tile must hold whole blocks");
 
   cg::cluster_group cluster = cg::this_cluster();
   const int K = L.K, R = L.R, m = L.m, n = L.n, T = L.T, tiles = L.tiles;
@@ -125,7 +128,6 @@ __global__ void __launch_bounds__(SOLVE_NT, 2) solve_kernel(const __grid_constan
   float* red = reinterpret_cast<float*>(smem + lay.red);
   double* slot = reinterpret_cast<double*>(smem + lay.slot);
   double* colsum = reinterpret_cast<double*>(smem + lay.colsum);
-  double* errv = reinterpret_cast<double*>(smem + lay.errv);
 
   auto code_at = [&](int row) -> uint32_t {
     if constexpr (SCB == 2) return reinterpret_cast<uint16_t*>(codes_v)[row * NBLK + bl];
@@ -180,53 +182,57 @@ __global__ void __launch_bounds__(SOLVE_NT, 2) solve_kernel(const __grid_constan
         bad |= !isfinite(__uint_as_float(v.x)) | !isfinite(__uint_as_float(v.y)) |
                !isfinite(__uint_as_float(v.z)) | !isfinite(__uint_as_float(v.w));
       }
-      const int P = row * S + part / ESZ, h = part % ESZ;
-      dst[chunk_pos<ESZ>(P, h)] = v;
+      dst[chunk_pos<ESZ>(row * S + part / CPP, part % CPP)] = v;
     }
     if (bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
   }
   __syncthreads();
 
-  float2 cc[8], ic[8];
+  float2 cc[4], ic[4];
   auto load_c = [&]() {
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      cc[p] = make_float2(cvec[s * 16 + 2 * p], cvec[s * 16 + 2 * p + 1]);
-      ic[p] = make_float2(icvec[s * 16 + 2 * p], icvec[s * 16 + 2 * p + 1]);
-    }
+    const float4* cv = reinterpret_cast<const float4*>(cvec + s * SEG);
+    const float4* iv = reinterpret_cast<const float4*>(icvec + s * SEG);
+    const float4 c0v = cv[0], c1v = cv[1], i0v = iv[0], i1v = iv[1];
+    cc[0] = make_float2(c0v.x, c0v.y); cc[1] = make_float2(c0v.z, c0v.w);
+    cc[2] = make_float2(c1v.x, c1v.y); cc[3] = make_float2(c1v.z, c1v.w);
+    ic[0] = make_float2(i0v.x, i0v.y); ic[1] = make_float2(i0v.z, i0v.w);
+    ic[2] = make_float2(i1v.x, i1v.y); ic[3] = make_float2(i1v.z, i1v.w);
   };
   load_c();
 
-  const int RPT = (R + NG - 1) / NG;
+  const int RPT = (Rc + NG - 1) / NG;        // uniform within the CTA (shuffles below)
   const int nh = n >> 1;
 
-  for (int t = 0; t <= T; ++t) {
-    const bool init = (t == 0);
-    const bool emit = (t == T);
-    float2 accN[8], accD[8], accS[8];
+  // One pass over the CTA's rows. INIT: iteration 0 (scales from absmax or r0, c = c0);
+  // otherwise one BCD iteration (Q-step, r-step + projection, c-step sums). EMIT: the
+  // returned state is written.
+  auto pass = [&](auto init_tag, auto emit_tag, const int t) {
+    constexpr bool INIT = decltype(init_tag)::value;
+    constexpr bool EMIT = decltype(emit_tag)::value;
+    float2 accN[4], accD[4], accS[INIT ? 4 : 1];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
+    for (int p = 0; p < 4; ++p) {
       accN[p] = make_float2(0.f, 0.f);
       accD[p] = make_float2(0.f, 0.f);
-      accS[p] = make_float2(0.f, 0.f);
+      if constexpr (INIT) accS[p] = make_float2(0.f, 0.f);
     }
 
     for (int k = 0; k < RPT; ++k) {
       const int row = g + k * NG;
       const bool valid = row < Rc;
-      float2 w[8];
+      float2 w[4];
       if (valid) {
         load_piece<ESZ>(Wsm, row * S + s, w);
       } else {
 #pragma unroll
-        for (int p = 0; p < 8; ++p) w[p] = make_float2(0.f, 0.f);
+        for (int p = 0; p < 4; ++p) w[p] = make_float2(0.f, 0.f);
       }
 
       ScaleVal sc;
-      if (init) {
+      if constexpr (INIT) {
         float a = 0.0f;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
+        for (int p = 0; p < 4; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
 #pragma unroll
         for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
         float v;
@@ -242,140 +248,181 @@ __global__ void __launch_bounds__(SOLVE_NT, 2) solve_kernel(const __grid_constan
       }
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
-      float2 q[8];
-      uint32_t cb[8];
+      float2 q[4];
+      uint32_t codes4 = 0;
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
-      for (int p = 0; p < 8; ++p) cb[p] = quant2<ELEM>(mul2(mul2(w[p], ic[p]), irr), q[p]);
+      for (int p = 0; p < 4; ++p) {
+        const uint32_t cb = quant2<ELEM>(mul2(mul2(w[p], ic[p]), irr), q[p]);
+        if constexpr (EMIT) codes4 |= cb << (8 * p);
+      }
 
-      if (!init) {
+      if constexpr (!INIT) {
         // r-step: least squares over the block, then projection
-        float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
+        if constexpr (SCALE == SCALE_BF16) {
+          // INT4's fine bf16 scale grid: block sums in binary64 keep projection decisions
+          // on the exact least-squares quotient
+          double num = 0.0, den = 0.0;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const float2 qc = mul2(q[p], cc[p]);
-          num2 = fma2(w[p], qc, num2);
-          den2 = fma2(qc, qc, den2);
-        }
-        float num = num2.x + num2.y, den = den2.x + den2.y;
+          for (int p = 0; p < 4; ++p) {
+            const double qcx = (double)q[p].x * (double)cc[p].x;
+            const double qcy = (double)q[p].y * (double)cc[p].y;
+            num = fma((double)w[p].x, qcx, num);
+            num = fma((double)w[p].y, qcy, num);
+            den = fma(qcx, qcx, den);
+            den = fma(qcy, qcy, den);
+          }
 #pragma unroll
-        for (int off = 1; off < LPB; off <<= 1) {
-          num += __shfl_xor_sync(FULL, num, off);
-          den += __shfl_xor_sync(FULL, den, off);
+          for (int off = 1; off < LPB; off <<= 1) {
+            num += __shfl_xor_sync(FULL, num, off);
+            den += __shfl_xor_sync(FULL, den, off);
+          }
+          if (den > 0.0) sc = project_scale<SCALE>(__double2float_rn(num / den), s_t, tbl);
+        } else {
+          float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 qc = mul2(q[p], cc[p]);
+            num2 = fma2(w[p], qc, num2);
+            den2 = fma2(qc, qc, den2);
+          }
+          float num = num2.x + num2.y, den = den2.x + den2.y;
+#pragma unroll
+          for (int off = 1; off < LPB; off <<= 1) {
+            num += __shfl_xor_sync(FULL, num, off);
+            den += __shfl_xor_sync(FULL, den, off);
+          }
+          if (den > 0.0f) sc = project_scale_ls<SCALE>(num, den, s_t, tbl);
         }
-        if (den > 0.0f) sc = project_scale<SCALE>(__fdiv_rn(num, den), s_t, tbl);
       }
       if (valid && lib == 0) set_code(row, sc.code);
 
       // c-step partial sums with the new r
       const float2 rr = make_float2(sc.r, sc.r);
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
+      for (int p = 0; p < 4; ++p) {
         const float2 qr = mul2(q[p], rr);
         accN[p] = fma2(w[p], qr, accN[p]);
         accD[p] = fma2(qr, qr, accD[p]);
-      }
-      if (init) {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) accS[p] = fma2(w[p], w[p], accS[p]);
+        if constexpr (INIT) accS[p] = fma2(w[p], w[p], accS[p]);
       }
 
-      if (emit && valid) {
-        const uint32_t lo = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
-        const uint32_t hi = cb[4] | (cb[5] << 8) | (cb[6] << 16) | (cb[7] << 24);
-        *reinterpret_cast<uint2*>(M.q_packed + (int64_t)(row0 + row) * nh + (col0 + s * 16) / 2) =
-            make_uint2(lo, hi);
-        if (lib == 0) {
-          const int64_t bi = (int64_t)(row0 + row) * nb + col0 / B + bl;
-          M.r[bi] = sc.r;
-          if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(M.bscale)[bi] = (uint16_t)sc.code;
-          else reinterpret_cast<uint8_t*>(M.bscale)[bi] = (uint8_t)sc.code;
+      if constexpr (EMIT) {
+        if (valid) {
+          *reinterpret_cast<uint32_t*>(M.q_packed + (int64_t)(row0 + row) * nh +
+                                       (col0 + s * SEG) / 2) = codes4;
+          if (lib == 0) {
+            const int64_t bi = (int64_t)(row0 + row) * nb + col0 / B + bl;
+            M.r[bi] = sc.r;
+            if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(M.bscale)[bi] = (uint16_t)sc.code;
+            else reinterpret_cast<uint8_t*>(M.bscale)[bi] = (uint8_t)sc.code;
+          }
         }
       }
     }
 
     // ---- per-column sums: warp (fp32) -> CTA (fp64) -> cluster (fp64, rank order)
     const int buf = t & 1;
-    double* myslot = slot + buf * 64 * S;
+    double* myslot = slot + buf * 32 * S;
     {
-      float v[32];
+      float v[16];
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
+      for (int p = 0; p < 4; ++p) {
         v[2 * p] = accN[p].x;
         v[2 * p + 1] = accN[p].y;
-        v[16 + 2 * p] = accD[p].x;
-        v[16 + 2 * p + 1] = accD[p].y;
+        v[8 + 2 * p] = accD[p].x;
+        v[8 + 2 * p + 1] = accD[p].y;
       }
       transpose_reduce<S>(v, lane);
 #pragma unroll
-      for (int i = 0; i < S; ++i) red[(warp * S + s) * 32 + (lane - s) + i] = v[i];
-      if (init) {
-        float u[32];
+      for (int i = 0; i < VPL; ++i) red[(warp * S + s) * 16 + (lane - s) / 2 + i] = v[i];
+      if constexpr (INIT) {
+        float u[16];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
+        for (int p = 0; p < 4; ++p) {
           u[2 * p] = accS[p].x;
           u[2 * p + 1] = accS[p].y;
-          u[16 + 2 * p] = 0.f;
-          u[16 + 2 * p + 1] = 0.f;
+          u[8 + 2 * p] = 0.f;
+          u[8 + 2 * p + 1] = 0.f;
         }
         transpose_reduce<S>(u, lane);
 #pragma unroll
-        for (int i = 0; i < S; ++i)
-          red[NWARP * S * 32 + (warp * S + s) * 32 + (lane - s) + i] = u[i];
+        for (int i = 0; i < VPL; ++i)
+          red[NWARP * S * 16 + (warp * S + s) * 16 + (lane - s) / 2 + i] = u[i];
       }
     }
     __syncthreads();
-    if (tid < 32 * S) {
-      double acc = 0.0, acs = 0.0;
-      for (int wp = 0; wp < NWARP; ++wp) acc += (double)red[wp * S * 32 + tid];
+    if (tid < 16 * S) {
+      double acc = 0.0;
+#pragma unroll
+      for (int wp = 0; wp < NWARP; ++wp) acc += (double)red[wp * S * 16 + tid];
       myslot[tid] = acc;
-      if (init) {
-        for (int wp = 0; wp < NWARP; ++wp) acs += (double)red[NWARP * S * 32 + wp * S * 32 + tid];
-        myslot[32 * S + tid] = acs;
+      if constexpr (INIT) {
+        double acs = 0.0;
+#pragma unroll
+        for (int wp = 0; wp < NWARP; ++wp) acs += (double)red[NWARP * S * 16 + wp * S * 16 + tid];
+        myslot[16 * S + tid] = acs;
       }
     }
     cluster.sync();
 
-    if (tid < TN) {
-      const int sj = tid >> 4, e = tid & 15;
-      double Nj = 0.0, Dj = 0.0, Sj = 0.0;
-      for (int rk = 0; rk < K; ++rk) {
-        const double* rs = cluster.map_shared_rank(myslot, rk);
-        Nj += rs[sj * 32 + e];
-        Dj += rs[sj * 32 + 16 + e];
-        if (init) Sj += rs[32 * S + sj * 32 + e];
+    // warp 0: per-column totals over the cluster (rank order), new c, error terms
+    double e = 0.0, q2 = 0.0;
+    if (warp == 0) {
+#pragma unroll
+      for (int jj = 0; jj < (TN + 31) / 32; ++jj) {
+        const int j = lane + 32 * jj;
+        if (j < TN) {
+          const int sj = j >> 3, ej = j & 7;
+          double Nj = 0.0, Dj = 0.0, Sj = 0.0;
+#pragma unroll
+          for (int rk = 0; rk < SOLVE_MAXK; ++rk) {
+            if (rk < K) {
+              const double* rs = cluster.map_shared_rank(myslot, rk);
+              Nj += rs[sj * 16 + ej];
+              Dj += rs[sj * 16 + 8 + ej];
+              if constexpr (INIT) Sj += rs[16 * S + sj * 16 + ej];
+            }
+          }
+          if constexpr (INIT) colsum[j] = Sj;
+          else Sj = colsum[j];
+          float cj = cvec[j];
+          if (!INIT && Dj > 0.0) {
+            cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
+            cvec[j] = cj;
+            icvec[j] = __frcp_rn(cj);
+          }
+          const double cd = (double)cj;
+          e += Sj - 2.0 * cd * Nj + cd * cd * Dj;
+          if constexpr (INIT) q2 += Sj;
+          if (EMIT && rank == 0) M.c[col0 + j] = cj;
+        }
       }
-      if (init) colsum[tid] = Sj;
-      else Sj = colsum[tid];
-      float cj = cvec[tid];
-      if (!init && Dj > 0.0) {
-        cj = __double2float_rn(Nj / Dj);
-        cvec[tid] = cj;
-        icvec[tid] = __frcp_rn(cj);
-      }
-      const double cd = (double)cj;
-      errv[tid] = Sj - 2.0 * cd * Nj + cd * cd * Dj;
-      if (emit && rank == 0) M.c[col0 + tid] = cj;
     }
     __syncthreads();
+    if constexpr (!INIT) load_c();
+    // trace terms of this tile (rank 0), off the other warps' critical path
     if (warp == 0 && rank == 0) {
-      double e = 0.0, q2 = 0.0;
-      for (int j = lane; j < TN; j += 32) {
-        e += errv[j];
-        if (init) q2 += colsum[j];
-      }
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) {
         e += __shfl_xor_sync(FULL, e, off);
-        q2 += __shfl_xor_sync(FULL, q2, off);
+        if constexpr (INIT) q2 += __shfl_xor_sync(FULL, q2, off);
       }
       if (lane == 0) {
         M.ws_err[(int64_t)t * tiles + tile] = e;
-        if (init) M.ws_wsq[tile] = q2;
+        if constexpr (INIT) M.ws_wsq[tile] = q2;
       }
     }
-    if (!init) load_c();
+  };
+
+  if (T == 0) {
+    pass(std::true_type{}, std::true_type{}, 0);
+  } else {
+    pass(std::true_type{}, std::false_type{}, 0);
+    for (int t = 1; t < T; ++t) pass(std::false_type{}, std::false_type{}, t);
+    pass(std::false_type{}, std::true_type{}, T);
   }
+
   // keep this CTA's slots alive until every CTA of the cluster has read them
   cluster.sync();
 }
@@ -475,48 +522,41 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ct
                 SolvePlan* p) {
   const int B = fmt_block(kind, group);
   if (B == 0 || m <= 0 || n <= 0 || n % B) return false;
-  const int LPB = B / 16;
-  // candidate segment counts, widest first
-  int cands[2] = {LPB, LPB};
-  int nc = 1;
-  if (kind == 3) { cands[0] = 2; cands[1] = 1; nc = 2; }       // NVFP4: 32 or 16 columns
-  else if (kind == 1 || kind == 2) { cands[0] = 2; nc = 1; }   // MX: 32 columns
-  for (int ci = 0; ci < nc; ++ci) {
-    const int S = cands[ci];
-    const int TN = 16 * S;
-    if (n % TN) continue;
-    const int64_t tiles = n / TN;
-    const int64_t slab = m * (int64_t)TN * esize;
-    int K = 1;
-    while ((int64_t)K * (int64_t)SOLVE_WTILE_MAX < slab) K <<= 1;
-    if (K > SOLVE_MAXK) continue;
-    // spread small problems over more SMs
-    while (K < SOLVE_MAXK && tiles * K * ctas_hint < 2 * 148 && (m + 2 * K - 1) / (2 * K) >= 16)
-      K <<= 1;
-    const int R = (int)((m + K - 1) / K);
-    const SolveSmem l = solve_smem(R, S, LPB, esize, kind == 0 ? 2 : 1);
-    if (l.total > 227 * 1024) continue;
-    p->S = S;
-    p->K = K;
-    p->R = R;
-    p->tiles = (int)tiles;
-    p->smem = l.total;
-    return true;
+  const int LPB = B / 8;
+  // the tile is one format block wide (NVFP4: 16, MX: 32, INT4: the group)
+  const int S = LPB;
+  const int TN = 8 * S;
+  const int64_t tiles = n / TN;
+  const int64_t slab = m * (int64_t)TN * esize;
+  int K = (int)std::max<int64_t>(1, (slab + (int64_t)SOLVE_WTILE_MAX - 1) / SOLVE_WTILE_MAX);
+  if (K > SOLVE_MAXK) {
+    // tall strips: the largest cluster with bigger tiles (fewer CTAs per SM)
+    K = SOLVE_MAXK;
+    if ((m + K - 1) / K * (int64_t)TN * esize > (int64_t)SOLVE_WTILE_BIG) return false;
   }
-  return false;
+  // spread small problems over more SMs
+  while (K < SOLVE_MAXK && tiles * K * ctas_hint < 3 * 148 && (m + 2 * K - 1) / (2 * K) >= 16)
+    K = std::min(SOLVE_MAXK, 2 * K);
+  const int R = (int)((m + K - 1) / K);
+  const SolveSmem l = solve_smem(R, S, LPB, esize, kind == 0 ? 2 : 1);
+  if (l.total > 227 * 1024) return false;
+  p->S = S;
+  p->K = K;
+  p->R = R;
+  p->tiles = (int)tiles;
+  p->smem = l.total;
+  return true;
 }
 
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s) {
   switch (kind) {
     case 0:
-      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4, 4>(L, count, esize, p, s);
-      return launch_dtype<ELEM_INT4, SCALE_BF16, 8, 8>(L, count, esize, p, s);
-    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
-    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
-    case 3:
-      if (p.S == 2) return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, 2>(L, count, esize, p, s);
-      return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, 1>(L, count, esize, p, s);
+      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 8, 8>(L, count, esize, p, s);
+      return launch_dtype<ELEM_INT4, SCALE_BF16, 16, 16>(L, count, esize, p, s);
+    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 4, 4>(L, count, esize, p, s);
+    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 4, 4>(L, count, esize, p, s);
+    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 2, 2>(L, count, esize, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
