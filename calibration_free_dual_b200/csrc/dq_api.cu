@@ -204,6 +204,7 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
       L.K = plan.K;
       L.R = plan.R;
       L.tiles = plan.tiles;
+      L.count = c;
       L.err_word = errp;
       for (int k = 0; k < c; ++k) {
         const int64_t idx = grp[base + k];

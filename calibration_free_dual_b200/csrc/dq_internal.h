@@ -10,8 +10,11 @@ namespace dq {
 constexpr int SOLVE_NT = 256;          // threads per CTA of the solve kernel
 constexpr int SOLVE_MAXMATS = 32;      // matrices per solve launch (descriptors by value)
 constexpr int SOLVE_MAXK = 8;          // CTAs per cluster (portable cluster size)
-constexpr size_t SOLVE_WTILE_MAX = 64 * 1024;    // preferred: 3 CTAs per SM
-constexpr size_t SOLVE_WTILE_BIG = 200 * 1024;   // ceiling for tall strips   // bytes of W kept per CTA
+constexpr int SOLVE_SEG = 16;          // columns of a row one thread owns
+// shared memory per CTA (everything, not just W) that lets 3 / 2 / 1 CTAs share an SM
+constexpr size_t SOLVE_SMEM_3PERSM = 72 * 1024;
+constexpr size_t SOLVE_SMEM_2PERSM = 110 * 1024;
+constexpr size_t SOLVE_SMEM_1PERSM = 227 * 1024;   // bytes of W kept per CTA
 
 struct SolveMat {
   const void* W;
@@ -29,13 +32,13 @@ struct SolveMat {
 };
 
 struct SolveLaunch {
-  int m, n, T, K, R, tiles;
+  int m, n, T, K, R, tiles, count;
   unsigned* err_word;
   SolveMat mats[SOLVE_MAXMATS];
 };
 
 struct SolvePlan {
-  int S;        // 8-column segments per CTA tile (tile width TN = 8*S)
+  int S;        // SOLVE_SEG-column segments per CTA tile (tile width TN = SOLVE_SEG*S)
   int K;        // CTAs per cluster (row split of one column strip)
   int R;        // rows per CTA
   int tiles;    // column tiles per matrix (n / TN)
@@ -44,13 +47,14 @@ struct SolvePlan {
 
 // Shared-memory carve-up of a solve CTA (same arithmetic on host and device).
 struct SolveSmem {
-  size_t w, codes, tbl, cvec, icvec, red, slot, colsum, errv, total;
+  size_t w, codes, tbl, cvec, icvec, red, slot, colsum, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize, int scb) {
-  const int TN = 8 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
+__host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize, int scb,
+                                                 int K, int SEG) {
+  const int TN = SEG * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32, NV = 2 * SEG;
   SolveSmem l;
   size_t off = 0;
   l.w = off;      off = align_up(off + (size_t)R * TN * esize, 128);
@@ -58,10 +62,9 @@ __host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize
   l.tbl = off;    off = align_up(off + 128 * 8, 16);
   l.cvec = off;   off = align_up(off + TN * 4, 16);
   l.icvec = off;  off = align_up(off + TN * 4, 16);
-  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * 16 * 4, 16);
-  l.slot = off;   off = align_up(off + (size_t)2 * 32 * S * 8, 16);
+  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * NV * 4, 16);
+  l.slot = off;   off = align_up(off + (size_t)2 * K * 2 * NV * S * 8, 16);
   l.colsum = off; off = align_up(off + TN * 8, 16);
-  l.errv = off;
   l.total = off;
   return l;
 }

@@ -22,7 +22,10 @@
 //   * one cluster barrier per iteration (double-buffered partial slots), no spin-waits.
 #include <cooperative_groups.h>
 
+#include <mutex>
 #include <type_traits>
+#include <utility>
+#include <vector>
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
@@ -33,33 +36,30 @@ namespace dq {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int SEG = 8;                 // columns per thread segment
 
-// 16-byte chunk position of chunk h of the 8-column piece P (row-major [R][TN] tile).
-// bf16: one chunk per piece, 8 lanes of a quarter warp read 128 contiguous bytes.
-// fp32: two chunks per piece, swizzled so a quarter warp hits 8 distinct bank groups.
-template <int ESZ>
+// 16-byte chunk position of chunk h of piece P (the SEG columns one thread owns in one row;
+// row-major [R][TN] tile, pieces of CPP chunks). The 8 lanes of a quarter warp read 8
+// consecutive pieces; the swizzle spreads them over the 8 bank groups.
+template <int CPP>
 __device__ __forceinline__ int chunk_pos(int P, int h) {
-  if constexpr (ESZ == 2) {
-    return P;
-  } else {
-    return 2 * P + (h ^ ((P >> 2) & 1));
-  }
+  if constexpr (CPP == 1) return P;
+  else if constexpr (CPP == 2) return 2 * P + (h ^ ((P >> 2) & 1));
+  else return 4 * P + (h ^ ((P >> 1) & 3));
 }
 
-template <int ESZ>
-__device__ __forceinline__ void load_piece(const unsigned char* Wsm, int P, float2 (&w)[4]) {
+template <int SEG, int ESZ>
+__device__ __forceinline__ void load_piece(const unsigned char* Wsm, int P, float2 (&w)[SEG / 2]) {
+  constexpr int CPP = SEG * ESZ / 16;
   const uint4* base = reinterpret_cast<const uint4*>(Wsm);
-  if constexpr (ESZ == 2) {
-    const uint4 v = base[chunk_pos<2>(P, 0)];
-    w[0] = bf16x2_to_f2(v.x);
-    w[1] = bf16x2_to_f2(v.y);
-    w[2] = bf16x2_to_f2(v.z);
-    w[3] = bf16x2_to_f2(v.w);
-  } else {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 v = base[chunk_pos<4>(P, h)];
+  for (int h = 0; h < CPP; ++h) {
+    const uint4 v = base[chunk_pos<CPP>(P, h)];
+    if constexpr (ESZ == 2) {
+      w[4 * h + 0] = bf16x2_to_f2(v.x);
+      w[4 * h + 1] = bf16x2_to_f2(v.y);
+      w[4 * h + 2] = bf16x2_to_f2(v.z);
+      w[4 * h + 3] = bf16x2_to_f2(v.w);
+    } else {
       w[2 * h + 0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
       w[2 * h + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
     }
@@ -73,17 +73,18 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// Butterfly reduction of a 16-value vector over the 32/S lanes sharing segment s = lane % S.
-// Lane L ends with S/2 consecutive values starting at index (L - s) / 2 (fixed order).
-template <int S>
-__device__ __forceinline__ void transpose_reduce(float (&v)[16], int lane) {
-  int cnt = 16;
+// Butterfly reduction of an NV-value vector over the 32/S lanes sharing segment
+// s = lane % S. Lane L ends with NV*S/32 consecutive values starting at (L - s)*NV/32
+// (fixed order: deterministic).
+template <int S, int NV>
+__device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane) {
+  int cnt = NV;
 #pragma unroll
   for (int off = 16; off >= S; off >>= 1) {
     const int half = cnt >> 1;
     const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < NV / 2; ++i) {
       if (i < half) {
         const float send = upper ? v[i] : v[i + half];
         const float keep = upper ? v[i + half] : v[i];
@@ -94,32 +95,36 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[16], int lane) {
   }
 }
 
-template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-__global__ void __launch_bounds__(SOLVE_NT, (SCALE == SCALE_BF16) ? 2 : 3)
+// One CTA: rows [rank*R, rank*R + R) of the column tile [tile*TN, tile*TN + TN) of matrix
+// blockIdx.y. Threads own SEG-column pieces of rows; LPB lanes share one format block.
+template <int ELEM, int SCALE, int SEG, int LPB, int S, bool F32IN>
+__global__ void __launch_bounds__(SOLVE_NT, 2)
 solve_kernel(const __grid_constant__ SolveLaunch L) {
   constexpr int NT = SOLVE_NT, NWARP = NT / 32, TN = SEG * S, NBLK = S / LPB, B = SEG * LPB;
   constexpr int NG = NT / S;            // rows covered by one pass of all threads
-  constexpr int VPL = S / 2;            // reduced values per lane
+  constexpr int NP = SEG / 2;           // float2 pairs per piece
+  constexpr int NV = 2 * SEG;           // per-thread column sums (N, D) of one pass
+  constexpr int VPL = NV * S / 32;      // reduced values per lane
   constexpr int ESZ = F32IN ? 4 : 2;
-  constexpr int CPP = ESZ / 2;          // 16-byte chunks per 8-column piece
+  constexpr int CPP = SEG * ESZ / 16;   // 16-byte chunks per piece
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
   constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
-  static_assert(NBLK * LPB == S && S >= 2 && S <= 16, "tile must hold whole blocks");
+  static_assert(NBLK * LPB == S && S >= 1 && S <= 8 && (SEG == 8 || SEG == 16), "tile shape");
 
   cg::cluster_group cluster = cg::this_cluster();
   const int K = L.K, R = L.R, m = L.m, n = L.n, T = L.T, tiles = L.tiles;
   const int rank = (int)cluster.block_rank();
-  const int tile = blockIdx.x / K;
-  const SolveMat& M = L.mats[blockIdx.y];
   const int row0 = rank * R;
   const int Rc = max(0, min(R, m - row0));
+  const int tile = blockIdx.x / K;
+  const SolveMat& M = L.mats[blockIdx.y];
   const int col0 = tile * TN;
   const int nb = n / B;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s = tid % S, g = tid / S, bl = s / LPB, lib = s % LPB;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const SolveSmem lay = solve_smem(R, S, LPB, ESZ, SCB);
+  const SolveSmem lay = solve_smem(R, S, LPB, ESZ, SCB, K, SEG);
   unsigned char* Wsm = smem + lay.w;
   void* codes_v = smem + lay.codes;
   float2* tbl = reinterpret_cast<float2*>(smem + lay.tbl);
@@ -182,21 +187,24 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         bad |= !isfinite(__uint_as_float(v.x)) | !isfinite(__uint_as_float(v.y)) |
                !isfinite(__uint_as_float(v.z)) | !isfinite(__uint_as_float(v.w));
       }
-      dst[chunk_pos<ESZ>(row * S + part / CPP, part % CPP)] = v;
+      dst[chunk_pos<CPP>(row * S + part / CPP, part % CPP)] = v;
     }
     if (bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
   }
   __syncthreads();
 
-  float2 cc[4], ic[4];
+  float2 cc[NP], ic[NP];
   auto load_c = [&]() {
     const float4* cv = reinterpret_cast<const float4*>(cvec + s * SEG);
     const float4* iv = reinterpret_cast<const float4*>(icvec + s * SEG);
-    const float4 c0v = cv[0], c1v = cv[1], i0v = iv[0], i1v = iv[1];
-    cc[0] = make_float2(c0v.x, c0v.y); cc[1] = make_float2(c0v.z, c0v.w);
-    cc[2] = make_float2(c1v.x, c1v.y); cc[3] = make_float2(c1v.z, c1v.w);
-    ic[0] = make_float2(i0v.x, i0v.y); ic[1] = make_float2(i0v.z, i0v.w);
-    ic[2] = make_float2(i1v.x, i1v.y); ic[3] = make_float2(i1v.z, i1v.w);
+#pragma unroll
+    for (int h = 0; h < SEG / 4; ++h) {
+      const float4 a = cv[h], b = iv[h];
+      cc[2 * h] = make_float2(a.x, a.y);
+      cc[2 * h + 1] = make_float2(a.z, a.w);
+      ic[2 * h] = make_float2(b.x, b.y);
+      ic[2 * h + 1] = make_float2(b.z, b.w);
+    }
   };
   load_c();
 
@@ -209,9 +217,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   auto pass = [&](auto init_tag, auto emit_tag, const int t) {
     constexpr bool INIT = decltype(init_tag)::value;
     constexpr bool EMIT = decltype(emit_tag)::value;
-    float2 accN[4], accD[4], accS[INIT ? 4 : 1];
+    float2 accN[NP], accD[NP], accS[INIT ? NP : 1];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
+    for (int p = 0; p < NP; ++p) {
       accN[p] = make_float2(0.f, 0.f);
       accD[p] = make_float2(0.f, 0.f);
       if constexpr (INIT) accS[p] = make_float2(0.f, 0.f);
@@ -220,19 +228,19 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     for (int k = 0; k < RPT; ++k) {
       const int row = g + k * NG;
       const bool valid = row < Rc;
-      float2 w[4];
+      float2 w[NP];
       if (valid) {
-        load_piece<ESZ>(Wsm, row * S + s, w);
+        load_piece<SEG, ESZ>(Wsm, row * S + s, w);
       } else {
 #pragma unroll
-        for (int p = 0; p < 4; ++p) w[p] = make_float2(0.f, 0.f);
+        for (int p = 0; p < NP; ++p) w[p] = make_float2(0.f, 0.f);
       }
 
       ScaleVal sc;
       if constexpr (INIT) {
         float a = 0.0f;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
+        for (int p = 0; p < NP; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
 #pragma unroll
         for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
         float v;
@@ -248,13 +256,15 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
-      float2 q[4];
-      uint32_t codes4 = 0;
+      float2 q[NP];
+      uint32_t codes[(NP + 3) / 4];
+#pragma unroll
+      for (int i = 0; i < (NP + 3) / 4; ++i) codes[i] = 0u;
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < NP; ++p) {
         const uint32_t cb = quant2<ELEM>(mul2(mul2(w[p], ic[p]), irr), q[p]);
-        if constexpr (EMIT) codes4 |= cb << (8 * p);
+        if constexpr (EMIT) codes[p >> 2] |= cb << (8 * (p & 3));
       }
 
       if constexpr (!INIT) {
@@ -264,7 +274,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
           // on the exact least-squares quotient
           double num = 0.0, den = 0.0;
 #pragma unroll
-          for (int p = 0; p < 4; ++p) {
+          for (int p = 0; p < NP; ++p) {
             const double qcx = (double)q[p].x * (double)cc[p].x;
             const double qcy = (double)q[p].y * (double)cc[p].y;
             num = fma((double)w[p].x, qcx, num);
@@ -281,7 +291,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         } else {
           float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int p = 0; p < 4; ++p) {
+          for (int p = 0; p < NP; ++p) {
             const float2 qc = mul2(q[p], cc[p]);
             num2 = fma2(w[p], qc, num2);
             den2 = fma2(qc, qc, den2);
@@ -300,7 +310,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       // c-step partial sums with the new r
       const float2 rr = make_float2(sc.r, sc.r);
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < NP; ++p) {
         const float2 qr = mul2(q[p], rr);
         accN[p] = fma2(w[p], qr, accN[p]);
         accD[p] = fma2(qr, qr, accD[p]);
@@ -309,8 +319,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
       if constexpr (EMIT) {
         if (valid) {
-          *reinterpret_cast<uint32_t*>(M.q_packed + (int64_t)(row0 + row) * nh +
-                                       (col0 + s * SEG) / 2) = codes4;
+          uint8_t* qp = M.q_packed + (int64_t)(row0 + row) * nh + (col0 + s * SEG) / 2;
+          if constexpr (NP == 8) *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
+          else *reinterpret_cast<uint32_t*>(qp) = codes[0];
           if (lib == 0) {
             const int64_t bi = (int64_t)(row0 + row) * nb + col0 / B + bl;
             M.r[bi] = sc.r;
@@ -323,45 +334,51 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
     // ---- per-column sums: warp (fp32) -> CTA (fp64) -> cluster (fp64, rank order)
     const int buf = t & 1;
-    double* myslot = slot + buf * 32 * S;
+    double* bufslot = slot + buf * K * 2 * NV * S;      // [K ranks][2 NV S] of this iteration
     {
-      float v[16];
+      float v[NV];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
+      for (int p = 0; p < NP; ++p) {
         v[2 * p] = accN[p].x;
         v[2 * p + 1] = accN[p].y;
-        v[8 + 2 * p] = accD[p].x;
-        v[8 + 2 * p + 1] = accD[p].y;
+        v[SEG + 2 * p] = accD[p].x;
+        v[SEG + 2 * p + 1] = accD[p].y;
       }
-      transpose_reduce<S>(v, lane);
+      transpose_reduce<S, NV>(v, lane);
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) red[(warp * S + s) * 16 + (lane - s) / 2 + i] = v[i];
+      for (int i = 0; i < VPL; ++i) red[(warp * S + s) * NV + (lane - s) * NV / 32 + i] = v[i];
       if constexpr (INIT) {
-        float u[16];
+        float u[NV];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
+        for (int p = 0; p < NP; ++p) {
           u[2 * p] = accS[p].x;
           u[2 * p + 1] = accS[p].y;
-          u[8 + 2 * p] = 0.f;
-          u[8 + 2 * p + 1] = 0.f;
+          u[SEG + 2 * p] = 0.f;
+          u[SEG + 2 * p + 1] = 0.f;
         }
-        transpose_reduce<S>(u, lane);
+        transpose_reduce<S, NV>(u, lane);
 #pragma unroll
         for (int i = 0; i < VPL; ++i)
-          red[NWARP * S * 16 + (warp * S + s) * 16 + (lane - s) / 2 + i] = u[i];
+          red[NWARP * S * NV + (warp * S + s) * NV + (lane - s) * NV / 32 + i] = u[i];
       }
     }
     __syncthreads();
-    if (tid < 16 * S) {
-      double acc = 0.0;
+    if (tid < NV * S) {
+      double acc = 0.0, acs = 0.0;
 #pragma unroll
-      for (int wp = 0; wp < NWARP; ++wp) acc += (double)red[wp * S * 16 + tid];
-      myslot[tid] = acc;
+      for (int wp = 0; wp < NWARP; ++wp) acc += (double)red[wp * S * NV + tid];
       if constexpr (INIT) {
-        double acs = 0.0;
 #pragma unroll
-        for (int wp = 0; wp < NWARP; ++wp) acs += (double)red[NWARP * S * 16 + wp * S * 16 + tid];
-        myslot[16 * S + tid] = acs;
+        for (int wp = 0; wp < NWARP; ++wp) acs += (double)red[NWARP * S * NV + wp * S * NV + tid];
+      }
+      // push this CTA's partial into row `rank` of every cluster peer's buffer
+#pragma unroll
+      for (int rk = 0; rk < SOLVE_MAXK; ++rk) {
+        if (rk < K) {
+          double* dst = cluster.map_shared_rank(bufslot, rk) + rank * 2 * NV * S;
+          dst[tid] = acc;
+          if constexpr (INIT) dst[NV * S + tid] = acs;
+        }
       }
     }
     cluster.sync();
@@ -373,15 +390,15 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       for (int jj = 0; jj < (TN + 31) / 32; ++jj) {
         const int j = lane + 32 * jj;
         if (j < TN) {
-          const int sj = j >> 3, ej = j & 7;
+          const int sj = j / SEG, ej = j % SEG;
           double Nj = 0.0, Dj = 0.0, Sj = 0.0;
 #pragma unroll
           for (int rk = 0; rk < SOLVE_MAXK; ++rk) {
             if (rk < K) {
-              const double* rs = cluster.map_shared_rank(myslot, rk);
-              Nj += rs[sj * 16 + ej];
-              Dj += rs[sj * 16 + 8 + ej];
-              if constexpr (INIT) Sj += rs[16 * S + sj * 16 + ej];
+              const double* rs = bufslot + rk * 2 * NV * S;
+              Nj += rs[sj * NV + ej];
+              Dj += rs[sj * NV + SEG + ej];
+              if constexpr (INIT) Sj += rs[NV * S + sj * NV + ej];
             }
           }
           if constexpr (INIT) colsum[j] = Sj;
@@ -423,7 +440,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     pass(std::false_type{}, std::true_type{}, T);
   }
 
-  // keep this CTA's slots alive until every CTA of the cluster has read them
+  // every peer has finished writing into and reading from this CTA's buffers
   cluster.sync();
 }
 
@@ -484,9 +501,74 @@ __global__ void finalize_kernel(const __grid_constant__ FinalizeArgs A) {
   if (lane == 0) A.mse[mat][t] = (w > 0.0) ? e / w : 0.0;
 }
 
+// Cluster size for a shape: among K >= the smallest that fits, the one with the most CTAs
+// resident at once (cluster placement inside a GPC makes some sizes pack worse), ties to the
+// smaller K; rows per CTA stay >= 32 once K exceeds the minimum. Depends on the shape and the
+// device only, so results do not depend on how many matrices share a launch.
+template <typename Kern>
+SolvePlan choose_cluster(Kern kern, const SolvePlan& base, int m, int esize, int LPB, int scb) {
+  struct Key { const void* k; int m, tiles; size_t smem; int dev; };
+  static std::mutex mu;
+  static std::vector<std::pair<Key, SolvePlan>> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const Key key{reinterpret_cast<const void*>(kern), m, base.tiles, base.smem, dev};
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    for (auto& e : cache)
+      if (e.first.k == key.k && e.first.m == m && e.first.tiles == key.tiles &&
+          e.first.smem == key.smem && e.first.dev == dev)
+        return e.second;
+  }
+  SolvePlan best = base;
+  int64_t best_ctas = -1;
+  for (int K = base.K; K <= SOLVE_MAXK; ++K) {
+    const int R = (m + K - 1) / K;
+    if (K > base.K && R < 32) break;
+    const SolveSmem l = solve_smem(R, base.S, LPB, esize, scb, K, SOLVE_SEG);
+    if (l.total > 227 * 1024) continue;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)l.total) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      continue;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(K * base.tiles), 1, 1);
+    cfg.blockDim = dim3(SOLVE_NT, 1, 1);
+    cfg.dynamicSmemBytes = l.total;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)K;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
+      (void)cudaGetLastError();
+      continue;
+    }
+    const int64_t ctas = (int64_t)K * std::min<int64_t>(active, base.tiles);
+    if (ctas > best_ctas) {
+      best_ctas = ctas;
+      best.K = K;
+      best.R = R;
+      best.smem = l.total;
+    }
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  cache.emplace_back(key, best);
+  return best;
+}
+
 template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-cudaError_t launch_one(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
-  auto kern = solve_kernel<ELEM, SCALE, LPB, S, F32IN>;
+cudaError_t launch_one(const SolveLaunch& L0, int count, const SolvePlan& p0, cudaStream_t st) {
+  auto kern = solve_kernel<ELEM, SCALE, SOLVE_SEG, LPB, S, F32IN>;
+  constexpr int ESZ = F32IN ? 4 : 2;
+  const SolvePlan p = choose_cluster(kern, p0, L0.m, ESZ, LPB, SCALE == SCALE_BF16 ? 2 : 1);
+  SolveLaunch L = L0;
+  L.K = p.K;
+  L.R = p.R;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)p.smem);
   if (e != cudaSuccess) return e;
@@ -520,43 +602,41 @@ cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const Solve
 
 bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ctas_hint,
                 SolvePlan* p) {
+  (void)ctas_hint;
   const int B = fmt_block(kind, group);
   if (B == 0 || m <= 0 || n <= 0 || n % B) return false;
-  const int LPB = B / 8;
+  const int LPB = B / SOLVE_SEG;
   // the tile is one format block wide (NVFP4: 16, MX: 32, INT4: the group)
   const int S = LPB;
-  const int TN = 8 * S;
-  const int64_t tiles = n / TN;
-  const int64_t slab = m * (int64_t)TN * esize;
-  int K = (int)std::max<int64_t>(1, (slab + (int64_t)SOLVE_WTILE_MAX - 1) / SOLVE_WTILE_MAX);
-  if (K > SOLVE_MAXK) {
-    // tall strips: the largest cluster with bigger tiles (fewer CTAs per SM)
-    K = SOLVE_MAXK;
-    if ((m + K - 1) / K * (int64_t)TN * esize > (int64_t)SOLVE_WTILE_BIG) return false;
+  const int scb = kind == 0 ? 2 : 1;
+  // smallest cluster whose CTAs fit two per SM (the register limit), else one
+  const size_t budgets[2] = {SOLVE_SMEM_2PERSM, SOLVE_SMEM_1PERSM};
+  for (size_t budget : budgets) {
+    for (int K = 1; K <= SOLVE_MAXK; ++K) {
+      const int R = (int)((m + K - 1) / K);
+      const SolveSmem l = solve_smem(R, S, LPB, esize, scb, K, SOLVE_SEG);
+      if (l.total <= budget) {
+        p->S = S;
+        p->K = K;
+        p->R = R;
+        p->tiles = (int)(n / (SOLVE_SEG * S));
+        p->smem = l.total;
+        return true;
+      }
+    }
   }
-  // spread small problems over more SMs
-  while (K < SOLVE_MAXK && tiles * K * ctas_hint < 3 * 148 && (m + 2 * K - 1) / (2 * K) >= 16)
-    K = std::min(SOLVE_MAXK, 2 * K);
-  const int R = (int)((m + K - 1) / K);
-  const SolveSmem l = solve_smem(R, S, LPB, esize, kind == 0 ? 2 : 1);
-  if (l.total > 227 * 1024) return false;
-  p->S = S;
-  p->K = K;
-  p->R = R;
-  p->tiles = (int)tiles;
-  p->smem = l.total;
-  return true;
+  return false;
 }
 
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s) {
   switch (kind) {
     case 0:
-      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 8, 8>(L, count, esize, p, s);
-      return launch_dtype<ELEM_INT4, SCALE_BF16, 16, 16>(L, count, esize, p, s);
-    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 4, 4>(L, count, esize, p, s);
-    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 4, 4>(L, count, esize, p, s);
-    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 2, 2>(L, count, esize, p, s);
+      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4, 4>(L, count, esize, p, s);
+      return launch_dtype<ELEM_INT4, SCALE_BF16, 8, 8>(L, count, esize, p, s);
+    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
+    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
+    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, 1>(L, count, esize, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
