@@ -13,6 +13,7 @@ DQ_ERR_NONFINITE, DQ_ERR_TIMEOUT, DQ_ERR_CUDA, DQ_ERR_UNSUPPORTED = 5, 6, 7, 8
 DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4 = 0, 1, 2, 3
 DQ_F32, DQ_BF16 = 0, 1
 DQ_CODEC_INT4, DQ_CODEC_E2M1, DQ_CODEC_E4M3, DQ_CODEC_E8M0, DQ_CODEC_BF16 = 0, 1, 2, 3, 4
+DQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
 class dq_format(ctypes.Structure):
@@ -37,6 +38,9 @@ SIGNATURES = {
     "dq_solve": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, dq_format, c_int32,
                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                            c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "dq_solve_noalloc": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, dq_format,
+                                   c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                   c_void_p, c_void_p, c_void_p, c_void_p]),
     "dq_act_quant_workspace_bytes": (c_size_t, [c_int64, c_int64, dq_format]),
     "dq_act_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, c_void_p,
                                dq_format, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,

@@ -113,6 +113,29 @@ DQ_API dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, in
                           float* tensor_scale, double* mse_trace, void* workspace,
                           size_t workspace_bytes, void* stream);
 
+/* Bytes of the fixed scratch array that dq_solve_noalloc uses (per device). */
+#define DQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/* dq_solve without a workspace argument, for callers that cannot allocate device memory
+ * (for example a host that hands all device memory to its own pool allocator and does not
+ * allow a library to call cudaMalloc or any other allocating routine). The DualQuant pages
+ * have no counterpart to this call; it exists only for such callers.
+ * Same arguments, semantics and outputs as dq_solve, minus workspace and workspace_bytes.
+ * Scratch: a fixed DQ_NOALLOC_SCRATCH_BYTES array inside libdq.so (held by every device
+ * that loads the library, until the process exits). The first call on a device looks up
+ * that array's device address (cudaGetSymbolAddress) with the device current; make that
+ * first call before any stream capture. The call allocates and frees nothing.
+ * Every call on a device shares the one array and leaves its contents behind; the call
+ * clears what must start at zero itself. Calls whose GPU work overlaps (different streams,
+ * or different host threads, on the same device) race on the array: serialise them.
+ * Returns DQ_ERR_WORKSPACE, before touching the device, when the shape and iteration count
+ * need more scratch than DQ_NOALLOC_SCRATCH_BYTES (dq_solve_workspace_bytes tells how much). */
+DQ_API dq_status dq_solve_noalloc(const void* W, int32_t dtype, int64_t m, int64_t n,
+                                  int64_t ldw, dq_format fmt, int32_t iters, const float* r0,
+                                  const float* c0, uint8_t* q_packed, float* r, float* c,
+                                  void* block_scales, float* tensor_scale, double* mse_trace,
+                                  void* stream);
+
 /* Largest m the solver handles for a given n, format and dtype (0 if the format is bad). */
 DQ_API int64_t dq_solve_max_rows(int64_t n, dq_format fmt, int32_t dtype);
 
