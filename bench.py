@@ -43,6 +43,37 @@ OPS_PER_ELEM_INIT = 8
 HBM_BYTES_PER_ELEM_ITER = 2.125
 
 
+KERNEL_SOURCES = ("dq_solve.cu", "dq_device.cuh", "dq_internal.h")
+PROFILE = os.path.join(ROOT, "profiles", "solve_kernel_8b_nvfp4_full.md")
+
+
+def profiled_traffic_per_elem():
+    """DRAM bytes per weight element per solve from the committed ncu summary, or None when
+    the solve kernel's sources have changed since that capture."""
+    import hashlib
+    if not os.path.exists(PROFILE):
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "calibration_free_dual_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    vals = {}
+    with open(PROFILE) as fh:
+        for line in fh:
+            if ":" in line and line.strip().split(":")[0] in ("source_sha256_16",
+                                                                "dram_bytes_per_elem_solve"):
+                k, v = line.strip().split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != h.hexdigest()[:16]:
+        return None
+    return float(vals["dram_bytes_per_elem_solve"])
+
+
+def workload_name(count: int, elems: int, T: int) -> str:
+    return ("Llama-3.1-8B-shaped layer set (%d matrices, %.3e bf16 weights per GPU), NVFP4, %d "
+            "BCD iterations + activation rescale/NVFP4 quant 8192x4096" % (count, elems, T))
+
+
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -179,7 +210,8 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "oracle sample: " + desc},
+        "config": {"workload": workload_name(len(cfg.layer_set()), cfg.elements(), cfg.iters),
+                   "sample": desc},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -298,8 +330,11 @@ def run_ours(args, world, rank, local):
     ops = args.steps * elems * (OPS_PER_ELEM_ITER * T + OPS_PER_ELEM_INIT)
     achieved = ops / (kern_ms * 1e-3) / 1e12 if kern_ms > 0 else None
     hbm_equiv = args.steps * elems * T * HBM_BYTES_PER_ELEM_ITER / (kern_ms * 1e-3) / 1e9
+    tpe = profiled_traffic_per_elem()
+    traffic = tpe * elems / per_step if tpe is not None else None        # bytes per launch
     roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tops/s",
-            "frac": achieved / alu_peak if achieved else None, "traffic": None,
+            "frac": achieved / alu_peak if achieved else None, "traffic": traffic,
+            "traffic_unit": "DRAM bytes per solve launch (ncu capture, layer-set average)",
             "peak_source": "148 SMs x 128 FP32 lanes x %.0f MHz (FMA = 1 op)" % sm_max,
             "kernel": "solve_kernel", "kernel_ms_per_step": kern_ms / args.steps,
             "launches_timed": used,
@@ -329,9 +364,7 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": "Llama-3.1-8B-shaped layer set (%d matrices, %.3e bf16 "
-                                   "weights per GPU), NVFP4, %d BCD iterations + activation "
-                                   "rescale/NVFP4 quant 8192x4096" % (count, elems, T),
+            "config": {"workload": workload_name(count, elems, T),
                        "full_model_solve_s": ms_step * 1e-3,
                        "l2": "inputs larger than L2 (%.1f GB of weights per step)"
                              % (elems * 2 / 1e9),

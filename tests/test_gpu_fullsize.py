@@ -1,0 +1,83 @@
+"""Full-size layer sets in the benchmark's launch configuration (B200).
+
+Each layer set is drawn on the device and solved with one dq_solve_batched call over all of
+its matrices, as bench.py does. Checked on every matrix: the trace is monotone (Theorem 1 (i)
+of the DualQuant paper, Figure 2 (b)) and ends below single-scale RTN, the NVFP4 tensor
+scale equals fl32(amax/2688), the decoded scales match their codes, c is finite and
+positive. Checked against the oracle: sampled column strips of blocks {0, L/2, L-1} (the
+solve of a strip is independent of the other strips, and the oracle solves it alone with
+the whole matrix's amax), and the full trace of one k_proj per set.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import formats as F
+from oracle import solver as S
+from tests._parity import CODE_MATCH, SCALE_MATCH, C_REL, MSE_REL, oracle_format, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dq():
+    import calibration_free_dual_b200 as pkg
+    return pkg
+
+
+def _strip_parity(W, h, fmt, j0, label):
+    """Oracle on columns [j0, j0+B) of W (device tensor) vs the GPU's outputs there."""
+    B = fmt.block
+    Ws = W[:, j0:j0 + B].float().cpu().numpy().astype(np.float64)
+    amax = float(W.float().abs().max()) if fmt.kind == "NVFP4" else None
+    ora = S.solve(Ws, fmt, 16, amax=amax)
+    codes = F.unpack_codes(h["q_packed"][:, j0 // 2:(j0 + B) // 2])
+    same_q = F.decode_elem(codes, fmt) == ora["q"]
+    same_q |= (F.decode_elem(codes, fmt) == 0) & (ora["q"] == 0)      # -0 vs +0
+    sc = h["block_scales"].view(np.uint16) if fmt.scale == "bf16" else h["block_scales"]
+    sc = sc[:, j0 // B].astype(np.int64)
+    same_r = sc == ora["r_codes"][:, 0].astype(np.int64)
+    c_rel = np.linalg.norm(h["c"][j0:j0 + B] - ora["c"]) / np.linalg.norm(ora["c"])
+    assert same_q.mean() >= CODE_MATCH, (label, same_q.mean())
+    assert same_r.mean() >= SCALE_MATCH, (label, same_r.mean())
+    assert np.all(np.abs(sc[~same_r] - ora["r_codes"][:, 0][~same_r].astype(np.int64)) <= 1), label
+    assert c_rel <= C_REL, (label, c_rel)
+
+
+@pytest.mark.parametrize("cid", [2, 3, 4])
+def test_layer_set_full_size(dq, cid):
+    cfg = wl.CONFIGS[cid]
+    fmt = oracle_format(cfg.fmt)
+    layer = cfg.layer_set()
+    Ws = [wl.weight_device(cfg, b, p) for b, p, _, _ in layer]
+    outs = dq.solve_batched(Ws, cfg.fmt, cfg.iters)
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    L = cfg.blocks
+    sample_blocks = {0, L // 2, L - 1}
+    rng = np.random.default_rng(cid)
+    for (b, p, m, n), W, o in zip(layer, Ws, outs):
+        mse = o["mse"].cpu().numpy()
+        label = f"cfg{cid}/b{b}/{wl.PROJ[p]}"
+        assert np.all(mse[1:] <= mse[:-1] * (1 + 1e-6)), (label, mse)
+        assert mse[-1] < mse[0], label
+        c = o["c"].cpu().numpy()
+        assert np.all(np.isfinite(c)) and np.all(c > 0), label
+        if fmt.kind == "NVFP4":
+            amax = W.float().abs().max().item()
+            assert o["tensor_scale"].item() == np.float32(np.float32(amax) / np.float32(2688.0))
+        if b in sample_blocks:
+            h = to_host(o)
+            sc = h["block_scales"].view(np.uint16) if fmt.scale == "bf16" else h["block_scales"]
+            s_t = h["tensor_scale"][0] if fmt.kind == "NVFP4" else None
+            np.testing.assert_array_equal(h["r"], F.decode_scale(sc, fmt, s_t))
+            for j0 in (0, int(rng.integers(1, n // fmt.block)) * fmt.block):
+                _strip_parity(W, h, fmt, j0, f"{label}/cols{j0}")
+    # full trace parity on block-0 k_proj
+    k0 = next(i for i, (b, p, _, _) in enumerate(layer) if b == 0 and p == 1)
+    ora = S.solve(Ws[k0].float().cpu().numpy().astype(np.float64), fmt, cfg.iters)
+    mse = outs[k0]["mse"].cpu().numpy()
+    np.testing.assert_allclose(mse, ora["mse"], rtol=MSE_REL)
+    del Ws, outs
+    torch.cuda.empty_cache()

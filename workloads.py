@@ -14,7 +14,8 @@ Recipe (shared by host and device generators):
   * outlier count = round-half-even(fraction * dim), at least 1, drawn without replacement
   * Student-t(4) scaled to std s uses scale s / sqrt(2) (Var t4 = 2); it is drawn as
     Z * sqrt(4 / V) with V = -2 log(U1 U2) (a chi-square with 4 degrees of freedom)
-  * Laplace(b) is drawn by inverse CDF from a uniform U in (-1/2, 1/2)
+  * Laplace(b) is drawn as b * (E1 - E2), E = -ln(1 - U) with U uniform in [0, 1) (both
+    exponentials are finite: 1 - U is in (0, 1])
 """
 from __future__ import annotations
 
@@ -119,8 +120,9 @@ def _host_base(rng: np.random.Generator, dist: str, scale: float, shape) -> np.n
         v = -2.0 * np.log(u1 * u2)
         return z * np.sqrt(4.0 / v) * (scale / math.sqrt(2.0))
     if dist == "laplace":
-        u = rng.random(shape) - 0.5
-        return -scale * np.sign(u) * np.log1p(-2.0 * np.abs(u))
+        e1 = -np.log(1.0 - rng.random(shape))
+        e2 = -np.log(1.0 - rng.random(shape))
+        return scale * (e1 - e2)
     raise ValueError(dist)
 
 
@@ -173,8 +175,9 @@ def _dev_base(g: torch.Generator, dist: str, scale: float, shape, device) -> tor
         v = -2.0 * torch.log(u1 * u2)
         return z * torch.sqrt(4.0 / v) * (scale / math.sqrt(2.0))
     if dist == "laplace":
-        u = torch.rand(shape, generator=g, device=device) - 0.5
-        return -scale * torch.sign(u) * torch.log1p(-2.0 * u.abs())
+        e1 = -torch.log(1.0 - torch.rand(shape, generator=g, device=device))
+        e2 = -torch.log(1.0 - torch.rand(shape, generator=g, device=device))
+        return scale * (e1 - e2)
     raise ValueError(dist)
 
 
