@@ -201,10 +201,10 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
       L.m = (int)ms[i];
       L.n = (int)ns[i];
       L.T = iters;
-      L.K = plan.K;
       L.R = plan.R;
       L.tiles = plan.tiles;
       L.count = c;
+      L.wide = 1;
       L.err_word = errp;
       for (int k = 0; k < c; ++k) {
         const int64_t idx = grp[base + k];
@@ -212,6 +212,8 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
         dq::SolveMat& sm = L.mats[k];
         sm.W = d.W;
         sm.ldw = d.ldw;
+        if ((reinterpret_cast<uintptr_t>(d.W) & 31u) != 0 || (d.ldw * esize) % 32 != 0)
+          L.wide = 0;
         sm.r0 = d.r0;
         sm.c0 = d.c0;
         sm.q_packed = d.q_packed;

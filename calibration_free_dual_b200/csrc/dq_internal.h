@@ -7,14 +7,9 @@
 
 namespace dq {
 
-constexpr int SOLVE_NT = 256;          // threads per CTA of the solve kernel
+constexpr int SOLVE_NT = 512;          // threads per CTA of the solve kernel (one CTA per SM)
 constexpr int SOLVE_MAXMATS = 32;      // matrices per solve launch (descriptors by value)
-constexpr int SOLVE_MAXK = 8;          // CTAs per cluster (portable cluster size)
-constexpr int SOLVE_SEG = 16;          // columns of a row one thread owns
-// shared memory per CTA (everything, not just W) that lets 3 / 2 / 1 CTAs share an SM
-constexpr size_t SOLVE_SMEM_3PERSM = 72 * 1024;
-constexpr size_t SOLVE_SMEM_2PERSM = 110 * 1024;
-constexpr size_t SOLVE_SMEM_1PERSM = 227 * 1024;   // bytes of W kept per CTA
+constexpr size_t SOLVE_SMEM_MAX = 227 * 1024;   // dynamic shared memory of one CTA
 
 struct SolveMat {
   const void* W;
@@ -32,39 +27,42 @@ struct SolveMat {
 };
 
 struct SolveLaunch {
-  int m, n, T, K, R, tiles, count;
+  int m, n, T;
+  int R;                       // rows of each column tile kept in shared memory
+  int tiles, count;
+  int wide;                    // every W base and row pitch 32-byte aligned (256-bit loads)
   unsigned* err_word;
   SolveMat mats[SOLVE_MAXMATS];
 };
 
 struct SolvePlan {
-  int S;        // SOLVE_SEG-column segments per CTA tile (tile width TN = SOLVE_SEG*S)
-  int K;        // CTAs per cluster (row split of one column strip)
-  int R;        // rows per CTA
+  int S;        // 16-column pieces per CTA tile (tile width TN = 16*S)
+  int R;        // rows of the tile resident in shared memory (the rest stream from L2)
   int tiles;    // column tiles per matrix (n / TN)
   size_t smem;  // dynamic shared memory per CTA
 };
 
-// Shared-memory carve-up of a solve CTA (same arithmetic on host and device).
+// Shared-memory carve-up of a solve CTA (same arithmetic on host and device): the resident
+// rows of W, the scale code of every (row, block) of the tile, the E4M3 table, c and 1/c,
+// the per-warp column partials and the per-column fp64 sums (N, D, ||W_j||^2, error).
 struct SolveSmem {
-  size_t w, codes, tbl, cvec, icvec, red, slot, colsum, total;
+  size_t w, codes, tbl, cvec, icvec, red, cols, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SolveSmem solve_smem(int R, int S, int LPB, int esize, int scb,
-                                                 int K, int SEG) {
-  const int TN = SEG * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32, NV = 2 * SEG;
+__host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, int esize,
+                                                 int scb) {
+  const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
   SolveSmem l;
   size_t off = 0;
   l.w = off;      off = align_up(off + (size_t)R * TN * esize, 128);
-  l.codes = off;  off = align_up(off + (size_t)R * NBLK * scb, 16);
+  l.codes = off;  off = align_up(off + (size_t)m * NBLK * scb, 16);
   l.tbl = off;    off = align_up(off + 128 * 8, 16);
   l.cvec = off;   off = align_up(off + TN * 4, 16);
   l.icvec = off;  off = align_up(off + TN * 4, 16);
-  l.red = off;    off = align_up(off + (size_t)2 * NWARP * S * NV * 4, 16);
-  l.slot = off;   off = align_up(off + (size_t)2 * K * 2 * NV * S * 8, 16);
-  l.colsum = off; off = align_up(off + TN * 8, 16);
+  l.red = off;    off = align_up(off + (size_t)NWARP * S * 32 * 4, 16);
+  l.cols = off;   off = align_up(off + (size_t)4 * TN * 8, 16);
   l.total = off;
   return l;
 }

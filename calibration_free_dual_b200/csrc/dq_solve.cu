@@ -1,4 +1,4 @@
-// dq_solve.cu — cluster-resident dual-scale BCD solve (sm_100a).
+// dq_solve.cu — dual-scale BCD solve, one column strip per CTA (sm_100a).
 //
 // Method: DualQuant ("DualQuant: Dual-scale Calibration-free Weight-and-Activation
 // Quantization for LLMs", Abstract): W ~ diag(r) Q diag(c) fitted by block coordinate
@@ -7,63 +7,84 @@
 // abstract of the same paper); the normalised-MSE trace of Figure 2 (b).
 //
 // B200 design. With r per (row, B-column block) and c per column, every step couples only
-// columns of one block (r-step) or rows of one column (c-step), so the solve decomposes
-// exactly into independent B-column strips. One thread-block cluster owns one tile of
-// TN = 16*S columns (whole blocks) and splits its m rows over K CTAs; each CTA copies its
-// rows x TN slab of W into shared memory once and runs every BCD iteration from there, so W
-// crosses HBM once per solve instead of once per iteration. Per iteration:
-//   * each thread owns one 16-column segment of a set of rows; LPB = B/16 neighbouring
-//     lanes share one block and combine its r-step sums with xor shuffles;
+// columns of one block (r-step) or rows of one column (c-step), so the solve splits exactly
+// into independent column strips. One CTA (512 threads, one per SM) owns a tile of
+// TN = 16*S columns and ALL m rows of it, so every reduction of the solve is CTA-local and
+// needs only __syncthreads:
+//   * the first R rows of the tile stay in shared memory for the whole solve (copied once
+//     from HBM); the remaining rows are read again from L2 on every pass with 256-bit loads
+//     marked evict-last (the streamed rows of all resident CTAs stay far below the 126 MB
+//     L2), the next row in flight while the current one is processed;
+//   * each thread owns one 16-column piece of a set of rows; LPB = B/16 neighbouring lanes
+//     share one format block and combine its r-step sums with xor shuffles;
 //   * Q-, r- and c-step run per row in registers with packed fp32x2 arithmetic
 //     (FMUL2/FFMA2) and the E2M1/E4M3 cvt instructions;
-//   * per-column sums N_j, D_j: transposed warp reduction (fp32), cross-warp sum (fp64),
-//     then every CTA of the cluster sums the K per-CTA partials from distributed shared
-//     memory in rank order (fp64), so all CTAs derive bit-identical c_j;
-//   * one cluster barrier per iteration (double-buffered partial slots), no spin-waits.
-#include <cooperative_groups.h>
-
-#include <mutex>
+//   * per pass, the per-column sums N_j, D_j go through a butterfly inside each warp (fp32)
+//     and a fixed binary64 tree across the 16 warps; the warps that own the tree also form
+//     the closed-form c_j and the pass's error terms. Two barriers per pass, no spin-waits.
+#include <algorithm>
 #include <type_traits>
-#include <utility>
-#include <vector>
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace dq {
 namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
+constexpr int NWARP = SOLVE_NT / 32;
 
-// 16-byte chunk position of chunk h of piece P (the SEG columns one thread owns in one row;
-// row-major [R][TN] tile, pieces of CPP chunks). The 8 lanes of a quarter warp read 8
+// 16-byte chunk position of chunk h of piece P (the 16 columns one thread owns in one row;
+// row-major [R][TN] tile, CPP chunks per piece). The 8 lanes of a quarter warp read 8
 // consecutive pieces; the swizzle spreads them over the 8 bank groups.
 template <int CPP>
 __device__ __forceinline__ int chunk_pos(int P, int h) {
-  if constexpr (CPP == 1) return P;
-  else if constexpr (CPP == 2) return 2 * P + (h ^ ((P >> 2) & 1));
+  if constexpr (CPP == 2) return 2 * P + (h ^ ((P >> 2) & 1));
   else return 4 * P + (h ^ ((P >> 1) & 3));
 }
 
-template <int SEG, int ESZ>
-__device__ __forceinline__ void load_piece(const unsigned char* Wsm, int P, float2 (&w)[SEG / 2]) {
-  constexpr int CPP = SEG * ESZ / 16;
+// One row piece as raw words (bf16: 8 words; fp32: 16 words).
+template <int ESZ>
+struct Raw {
+  uint32_t u[ESZ * 4];
+};
+
+template <int ESZ>
+__device__ __forceinline__ void unpack(const Raw<ESZ>& r, float2 (&w)[8]) {
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    if constexpr (ESZ == 2) w[p] = bf16x2_to_f2(r.u[p]);
+    else w[p] = make_float2(__uint_as_float(r.u[2 * p]), __uint_as_float(r.u[2 * p + 1]));
+  }
+}
+
+template <int ESZ>
+__device__ __forceinline__ void zero(Raw<ESZ>& r) {
+#pragma unroll
+  for (int i = 0; i < ESZ * 4; ++i) r.u[i] = 0u;
+}
+
+template <int ESZ>
+__device__ __forceinline__ void load_smem(const unsigned char* Wsm, int P, Raw<ESZ>& r) {
   const uint4* base = reinterpret_cast<const uint4*>(Wsm);
 #pragma unroll
-  for (int h = 0; h < CPP; ++h) {
-    const uint4 v = base[chunk_pos<CPP>(P, h)];
-    if constexpr (ESZ == 2) {
-      w[4 * h + 0] = bf16x2_to_f2(v.x);
-      w[4 * h + 1] = bf16x2_to_f2(v.y);
-      w[4 * h + 2] = bf16x2_to_f2(v.z);
-      w[4 * h + 3] = bf16x2_to_f2(v.w);
-    } else {
-      w[2 * h + 0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
-      w[2 * h + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
-    }
+  for (int h = 0; h < ESZ; ++h) {
+    const uint4 v = base[chunk_pos<ESZ>(P, h)];
+    r.u[4 * h + 0] = v.x;
+    r.u[4 * h + 1] = v.y;
+    r.u[4 * h + 2] = v.z;
+    r.u[4 * h + 3] = v.w;
   }
+}
+
+// 32 bytes from L2, not allocated in L1, kept in L2 ahead of normal lines (evict-last):
+// these rows are read again on every pass.
+__device__ __forceinline__ void ldg256_keep(const void* p, uint32_t* d) {
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::evict_last.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
+        "=r"(d[7])
+      : "l"(p));
 }
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
@@ -73,18 +94,42 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return v;
 }
 
-// Butterfly reduction of an NV-value vector over the 32/S lanes sharing segment
-// s = lane % S. Lane L ends with NV*S/32 consecutive values starting at (L - s)*NV/32
-// (fixed order: deterministic).
-template <int S, int NV>
-__device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane) {
-  int cnt = NV;
+// A streamed row piece: 256-bit loads when every row start is 32-byte aligned, else 128-bit.
+template <int ESZ>
+__device__ __forceinline__ void load_global(const char* p, bool wide, Raw<ESZ>& r) {
+  if (wide) {
+#pragma unroll
+    for (int h = 0; h < ESZ / 2; ++h) ldg256_keep(p + 32 * h, r.u + 8 * h);
+  } else {
+#pragma unroll
+    for (int h = 0; h < ESZ; ++h) {
+      const uint4 v = ldg_stream(p + 16 * h);
+      r.u[4 * h + 0] = v.x;
+      r.u[4 * h + 1] = v.y;
+      r.u[4 * h + 2] = v.z;
+      r.u[4 * h + 3] = v.w;
+    }
+  }
+}
+
+__device__ __forceinline__ bool nonfinite8(const float2 (&w)[8]) {
+  bool bad = false;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) bad |= !isfinite(w[p].x) | !isfinite(w[p].y);
+  return bad;
+}
+
+// Butterfly reduction of 32 values over the 32/S lanes sharing piece s = lane % S.
+// Lane L ends with the S totals of indices [L - s, L - s + S) (fixed order).
+template <int S>
+__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
+  int cnt = 32;
 #pragma unroll
   for (int off = 16; off >= S; off >>= 1) {
     const int half = cnt >> 1;
     const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < NV / 2; ++i) {
+    for (int i = 0; i < 16; ++i) {
       if (i < half) {
         const float send = upper ? v[i] : v[i + half];
         const float keep = upper ? v[i + half] : v[i];
@@ -95,44 +140,38 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[NV], int lane) {
   }
 }
 
-// One CTA: rows [rank*R, rank*R + R) of the column tile [tile*TN, tile*TN + TN) of matrix
-// blockIdx.y. Threads own SEG-column pieces of rows; LPB lanes share one format block.
-template <int ELEM, int SCALE, int SEG, int LPB, int S, bool F32IN>
-__global__ void __launch_bounds__(SOLVE_NT, 2)
+// One CTA: all m rows of the column tile [tile*TN, tile*TN + TN) of matrix blockIdx.y.
+template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
+__global__ void __launch_bounds__(SOLVE_NT, 1)
 solve_kernel(const __grid_constant__ SolveLaunch L) {
-  constexpr int NT = SOLVE_NT, NWARP = NT / 32, TN = SEG * S, NBLK = S / LPB, B = SEG * LPB;
-  constexpr int NG = NT / S;            // rows covered by one pass of all threads
-  constexpr int NP = SEG / 2;           // float2 pairs per piece
-  constexpr int NV = 2 * SEG;           // per-thread column sums (N, D) of one pass
-  constexpr int VPL = NV * S / 32;      // reduced values per lane
+  constexpr int NT = SOLVE_NT, TN = 16 * S, NBLK = S / LPB, B = 16 * LPB;
+  constexpr int NG = NT / S;             // rows covered by one sweep of all threads
   constexpr int ESZ = F32IN ? 4 : 2;
-  constexpr int CPP = SEG * ESZ / 16;   // 16-byte chunks per piece
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
   constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
-  static_assert(NBLK * LPB == S && S >= 1 && S <= 8 && (SEG == 8 || SEG == 16), "tile shape");
+  static_assert(NBLK * LPB == S && S >= 1 && S <= 8, "tile shape");
 
-  cg::cluster_group cluster = cg::this_cluster();
-  const int K = L.K, R = L.R, m = L.m, n = L.n, T = L.T, tiles = L.tiles;
-  const int rank = (int)cluster.block_rank();
-  const int row0 = rank * R;
-  const int Rc = max(0, min(R, m - row0));
-  const int tile = blockIdx.x / K;
+  const int m = L.m, n = L.n, T = L.T, tiles = L.tiles;
+  const int tile = blockIdx.x;
   const SolveMat& M = L.mats[blockIdx.y];
   const int col0 = tile * TN;
   const int nb = n / B;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s = tid % S, g = tid / S, bl = s / LPB, lib = s % LPB;
+  const bool wide = L.wide != 0;
+  const char* gW = reinterpret_cast<const char*>(M.W) + (int64_t)(col0 + s * 16) * ESZ;
+  const int64_t pitch = M.ldw * ESZ;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const SolveSmem lay = solve_smem(R, S, LPB, ESZ, SCB, K, SEG);
+  const SolveSmem lay = solve_smem(m, L.R, S, LPB, ESZ, SCB);
   unsigned char* Wsm = smem + lay.w;
   void* codes_v = smem + lay.codes;
   float2* tbl = reinterpret_cast<float2*>(smem + lay.tbl);
   float* cvec = reinterpret_cast<float*>(smem + lay.cvec);
   float* icvec = reinterpret_cast<float*>(smem + lay.icvec);
   float* red = reinterpret_cast<float*>(smem + lay.red);
-  double* slot = reinterpret_cast<double*>(smem + lay.slot);
-  double* colsum = reinterpret_cast<double*>(smem + lay.colsum);
+  double* errw = reinterpret_cast<double*>(smem + lay.cols);   // [S] per-warp error sums
+  double* wsqw = errw + 8;                                     // [S] per-warp ||W||^2 sums
 
   auto code_at = [&](int row) -> uint32_t {
     if constexpr (SCB == 2) return reinterpret_cast<uint16_t*>(codes_v)[row * NBLK + bl];
@@ -152,7 +191,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       const float r = __fmul_rn(s_t, e4m3_decode(code));
       tbl[tid] = make_float2(r, __frcp_rn(r));
     }
-    if (tile == 0 && rank == 0 && tid == 0 && M.tensor_scale != nullptr) *M.tensor_scale = s_t;
+    if (tile == 0 && tid == 0 && M.tensor_scale != nullptr) *M.tensor_scale = s_t;
   }
 
   // ---- column scales: c0 or 1
@@ -169,36 +208,36 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     icvec[tid] = __frcp_rn(cj);
   }
 
-  // ---- copy this CTA's rows x TN slab of W into shared memory (the only read of W)
+  // ---- rows [0, min(R, m)) into shared memory (their only read from HBM)
   {
     constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
-    const char* gW = reinterpret_cast<const char*>(M.W);
-    const int64_t ldw = M.ldw;
+    const int rows = min(L.R, m);
+    const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
     uint4* dst = reinterpret_cast<uint4*>(Wsm);
     bool bad = false;
 #pragma unroll 4
-    for (int ch = tid; ch < Rc * CH; ch += NT) {
+    for (int ch = tid; ch < rows * CH; ch += NT) {
       const int row = ch / CH, part = ch % CH;
-      const uint4 v = ldg_stream(gW + ((int64_t)(row0 + row) * ldw + col0) * ESZ + part * 16);
+      const uint4 v = ldg_stream(base + (int64_t)row * pitch + part * 16);
       if constexpr (ESZ == 2) {
         bad |= bf16x2_nonfinite(v.x) | bf16x2_nonfinite(v.y) | bf16x2_nonfinite(v.z) |
                bf16x2_nonfinite(v.w);
       } else {
-        bad |= !isfinite(__uint_as_float(v.x)) | !isfinite(__uint_as_float(v.y)) |
-               !isfinite(__uint_as_float(v.z)) | !isfinite(__uint_as_float(v.w));
+        bad |= ((v.x & 0x7F800000u) == 0x7F800000u) | ((v.y & 0x7F800000u) == 0x7F800000u) |
+               ((v.z & 0x7F800000u) == 0x7F800000u) | ((v.w & 0x7F800000u) == 0x7F800000u);
       }
-      dst[chunk_pos<CPP>(row * S + part / CPP, part % CPP)] = v;
+      dst[chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ)] = v;
     }
     if (bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
   }
   __syncthreads();
 
-  float2 cc[NP], ic[NP];
+  float2 cc[8], ic[8];
   auto load_c = [&]() {
-    const float4* cv = reinterpret_cast<const float4*>(cvec + s * SEG);
-    const float4* iv = reinterpret_cast<const float4*>(icvec + s * SEG);
+    const float4* cv = reinterpret_cast<const float4*>(cvec + s * 16);
+    const float4* iv = reinterpret_cast<const float4*>(icvec + s * 16);
 #pragma unroll
-    for (int h = 0; h < SEG / 4; ++h) {
+    for (int h = 0; h < 4; ++h) {
       const float4 a = cv[h], b = iv[h];
       cc[2 * h] = make_float2(a.x, a.y);
       cc[2 * h + 1] = make_float2(a.z, a.w);
@@ -208,44 +247,87 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   };
   load_c();
 
-  const int RPT = (Rc + NG - 1) / NG;        // uniform within the CTA (shuffles below)
+  const int RPT = (m + NG - 1) / NG;       // sweeps per pass (uniform: shuffles below)
+  const int KS = min(L.R / NG, RPT);       // sweeps served from shared memory
   const int nh = n >> 1;
 
-  // One pass over the CTA's rows. INIT: iteration 0 (scales from absmax or r0, c = c0);
-  // otherwise one BCD iteration (Q-step, r-step + projection, c-step sums). EMIT: the
+  // row piece of sweep k: shared memory, L2, or zeros past the last row
+  auto fetch = [&](int k, Raw<ESZ>& dst) {
+    const int row = g + k * NG;
+    if (row >= m) zero<ESZ>(dst);
+    else if (k < KS) load_smem<ESZ>(Wsm, row * S + s, dst);
+    else load_global<ESZ>(gW + (int64_t)row * pitch, wide, dst);
+  };
+
+  // per-column totals of the 32-value vectors (a: 16 columns, b: 16 columns) of all
+  // threads; thread tid < 32*S (lane e of warp sj) returns the total of value e of piece sj
+  auto column_totals = [&](const float2 (&a)[8], const float2 (&b)[8]) -> double {
+    float v[32];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      v[2 * p] = a[p].x;
+      v[2 * p + 1] = a[p].y;
+      v[16 + 2 * p] = b[p].x;
+      v[16 + 2 * p + 1] = b[p].y;
+    }
+    transpose_reduce<S>(v, lane);
+#pragma unroll
+    for (int i = 0; i < S; ++i) red[(warp * S + s) * 32 + (lane - s) + i] = v[i];
+    __syncthreads();
+    double tot = 0.0;
+    if (tid < 32 * S) {
+      double va[NWARP];
+#pragma unroll
+      for (int wp = 0; wp < NWARP; ++wp) va[wp] = (double)red[wp * S * 32 + tid];
+#pragma unroll
+      for (int st = 1; st < NWARP; st <<= 1) {
+#pragma unroll
+        for (int i = 0; i + st < NWARP; i += 2 * st) va[i] += va[i + st];
+      }
+      tot = va[0];
+    }
+    return tot;
+  };
+
+  double Sj = 0.0;          // ||W_j||^2 of column sj*16 + lane (threads tid < 32*S, lane < 16)
+
+  // One pass over all rows of the tile. INIT: iteration 0 (scales from absmax or r0,
+  // c = c0); otherwise one BCD iteration (Q-step, r-step + projection, c-step). EMIT: the
   // returned state is written.
   auto pass = [&](auto init_tag, auto emit_tag, const int t) {
     constexpr bool INIT = decltype(init_tag)::value;
     constexpr bool EMIT = decltype(emit_tag)::value;
-    float2 accN[NP], accD[NP], accS[INIT ? NP : 1];
+    float2 accN[8], accD[8], accS[INIT ? 8 : 1];
 #pragma unroll
-    for (int p = 0; p < NP; ++p) {
+    for (int p = 0; p < 8; ++p) {
       accN[p] = make_float2(0.f, 0.f);
       accD[p] = make_float2(0.f, 0.f);
       if constexpr (INIT) accS[p] = make_float2(0.f, 0.f);
     }
+    bool bad = false;
 
+    Raw<ESZ> buf;
+    fetch(0, buf);
     for (int k = 0; k < RPT; ++k) {
       const int row = g + k * NG;
-      const bool valid = row < Rc;
-      float2 w[NP];
-      if (valid) {
-        load_piece<SEG, ESZ>(Wsm, row * S + s, w);
-      } else {
-#pragma unroll
-        for (int p = 0; p < NP; ++p) w[p] = make_float2(0.f, 0.f);
+      const bool valid = row < m;
+      float2 w[8];
+      unpack<ESZ>(buf, w);
+      if (k + 1 < RPT) fetch(k + 1, buf);
+      if constexpr (INIT) {
+        if (k >= KS) bad |= nonfinite8(w);
       }
 
       ScaleVal sc;
       if constexpr (INIT) {
         float a = 0.0f;
 #pragma unroll
-        for (int p = 0; p < NP; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
+        for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
 #pragma unroll
         for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
         float v;
         if (M.r0 != nullptr) {
-          v = valid ? M.r0[(int64_t)(row0 + row) * nb + col0 / B + bl] : 1.0f;
+          v = valid ? M.r0[(int64_t)row * nb + col0 / B + bl] : 1.0f;
         } else {
           v = (a > 0.0f) ? __fdiv_rn(a, QMAX) : 1.0f;
         }
@@ -256,13 +338,11 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
-      float2 q[NP];
-      uint32_t codes[(NP + 3) / 4];
-#pragma unroll
-      for (int i = 0; i < (NP + 3) / 4; ++i) codes[i] = 0u;
+      float2 q[8];
+      uint32_t codes[2] = {0u, 0u};
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
+      for (int p = 0; p < 8; ++p) {
         const uint32_t cb = quant2<ELEM>(mul2(mul2(w[p], ic[p]), irr), q[p]);
         if constexpr (EMIT) codes[p >> 2] |= cb << (8 * (p & 3));
       }
@@ -274,7 +354,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
           // on the exact least-squares quotient
           double num = 0.0, den = 0.0;
 #pragma unroll
-          for (int p = 0; p < NP; ++p) {
+          for (int p = 0; p < 8; ++p) {
             const double qcx = (double)q[p].x * (double)cc[p].x;
             const double qcy = (double)q[p].y * (double)cc[p].y;
             num = fma((double)w[p].x, qcx, num);
@@ -291,7 +371,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         } else {
           float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int p = 0; p < NP; ++p) {
+          for (int p = 0; p < 8; ++p) {
             const float2 qc = mul2(q[p], cc[p]);
             num2 = fma2(w[p], qc, num2);
             den2 = fma2(qc, qc, den2);
@@ -310,7 +390,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       // c-step partial sums with the new r
       const float2 rr = make_float2(sc.r, sc.r);
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
+      for (int p = 0; p < 8; ++p) {
         const float2 qr = mul2(q[p], rr);
         accN[p] = fma2(w[p], qr, accN[p]);
         accD[p] = fma2(qr, qr, accD[p]);
@@ -319,11 +399,10 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
       if constexpr (EMIT) {
         if (valid) {
-          uint8_t* qp = M.q_packed + (int64_t)(row0 + row) * nh + (col0 + s * SEG) / 2;
-          if constexpr (NP == 8) *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
-          else *reinterpret_cast<uint32_t*>(qp) = codes[0];
+          uint8_t* qp = M.q_packed + (int64_t)row * nh + (col0 + s * 16) / 2;
+          *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
           if (lib == 0) {
-            const int64_t bi = (int64_t)(row0 + row) * nb + col0 / B + bl;
+            const int64_t bi = (int64_t)row * nb + col0 / B + bl;
             M.r[bi] = sc.r;
             if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(M.bscale)[bi] = (uint16_t)sc.code;
             else reinterpret_cast<uint8_t*>(M.bscale)[bi] = (uint8_t)sc.code;
@@ -331,104 +410,57 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         }
       }
     }
+    if (INIT && bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
 
-    // ---- per-column sums: warp (fp32) -> CTA (fp64) -> cluster (fp64, rank order)
-    const int buf = t & 1;
-    double* bufslot = slot + buf * K * 2 * NV * S;      // [K ranks][2 NV S] of this iteration
-    {
-      float v[NV];
+    // ---- column sums (iteration 0 first forms ||W_j||^2, kept by its owner thread)
+    if constexpr (INIT) {
+      float2 zero2[8];
 #pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        v[2 * p] = accN[p].x;
-        v[2 * p + 1] = accN[p].y;
-        v[SEG + 2 * p] = accD[p].x;
-        v[SEG + 2 * p + 1] = accD[p].y;
-      }
-      transpose_reduce<S, NV>(v, lane);
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) red[(warp * S + s) * NV + (lane - s) * NV / 32 + i] = v[i];
-      if constexpr (INIT) {
-        float u[NV];
-#pragma unroll
-        for (int p = 0; p < NP; ++p) {
-          u[2 * p] = accS[p].x;
-          u[2 * p + 1] = accS[p].y;
-          u[SEG + 2 * p] = 0.f;
-          u[SEG + 2 * p + 1] = 0.f;
-        }
-        transpose_reduce<S, NV>(u, lane);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i)
-          red[NWARP * S * NV + (warp * S + s) * NV + (lane - s) * NV / 32 + i] = u[i];
-      }
+      for (int p = 0; p < 8; ++p) zero2[p] = make_float2(0.f, 0.f);
+      Sj = column_totals(accS, zero2);
+      __syncthreads();                       // the reduction buffer is reused
     }
-    __syncthreads();
-    if (tid < NV * S) {
-      double acc = 0.0, acs = 0.0;
-#pragma unroll
-      for (int wp = 0; wp < NWARP; ++wp) acc += (double)red[wp * S * NV + tid];
-      if constexpr (INIT) {
-#pragma unroll
-        for (int wp = 0; wp < NWARP; ++wp) acs += (double)red[NWARP * S * NV + wp * S * NV + tid];
-      }
-      // push this CTA's partial into row `rank` of every cluster peer's buffer
-#pragma unroll
-      for (int rk = 0; rk < SOLVE_MAXK; ++rk) {
-        if (rk < K) {
-          double* dst = cluster.map_shared_rank(bufslot, rk) + rank * 2 * NV * S;
-          dst[tid] = acc;
-          if constexpr (INIT) dst[NV * S + tid] = acs;
-        }
-      }
-    }
-    cluster.sync();
+    const double nd = column_totals(accN, accD);
 
-    // warp 0: per-column totals over the cluster (rank order), new c, error terms
-    double e = 0.0, q2 = 0.0;
-    if (warp == 0) {
-#pragma unroll
-      for (int jj = 0; jj < (TN + 31) / 32; ++jj) {
-        const int j = lane + 32 * jj;
-        if (j < TN) {
-          const int sj = j / SEG, ej = j % SEG;
-          double Nj = 0.0, Dj = 0.0, Sj = 0.0;
-#pragma unroll
-          for (int rk = 0; rk < SOLVE_MAXK; ++rk) {
-            if (rk < K) {
-              const double* rs = bufslot + rk * 2 * NV * S;
-              Nj += rs[sj * NV + ej];
-              Dj += rs[sj * NV + SEG + ej];
-              if constexpr (INIT) Sj += rs[NV * S + sj * NV + ej];
-            }
-          }
-          if constexpr (INIT) colsum[j] = Sj;
-          else Sj = colsum[j];
-          float cj = cvec[j];
-          if (!INIT && Dj > 0.0) {
-            cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
-            cvec[j] = cj;
-            icvec[j] = __frcp_rn(cj);
-          }
-          const double cd = (double)cj;
-          e += Sj - 2.0 * cd * Nj + cd * cd * Dj;
-          if constexpr (INIT) q2 += Sj;
-          if (EMIT && rank == 0) M.c[col0 + j] = cj;
+    // ---- c-step (closed form) and this pass's error terms: warps 0..S-1, lanes 0..15
+    if (tid < 32 * S) {
+      const double Dj = __shfl_down_sync(FULL, nd, 16);
+      double e = 0.0, q2 = 0.0;
+      if (lane < 16) {
+        const int j = warp * 16 + lane;
+        const double Nj = nd;
+        float cj = cvec[j];
+        if (!INIT && Dj > 0.0) {
+          cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
+          cvec[j] = cj;
+          icvec[j] = __frcp_rn(cj);
         }
+        if (EMIT) M.c[col0 + j] = cj;
+        const double cd = (double)cj;
+        e = Sj - 2.0 * cd * Nj + cd * cd * Dj;
+        if constexpr (INIT) q2 = Sj;
       }
-    }
-    __syncthreads();
-    if constexpr (!INIT) load_c();
-    // trace terms of this tile (rank 0), off the other warps' critical path
-    if (warp == 0 && rank == 0) {
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) {
         e += __shfl_xor_sync(FULL, e, off);
         if constexpr (INIT) q2 += __shfl_xor_sync(FULL, q2, off);
       }
       if (lane == 0) {
-        M.ws_err[(int64_t)t * tiles + tile] = e;
-        if constexpr (INIT) M.ws_wsq[tile] = q2;
+        errw[warp] = e;
+        if constexpr (INIT) wsqw[warp] = q2;
       }
+    }
+    __syncthreads();
+    if constexpr (!INIT) load_c();
+    if (tid == 0) {
+      double e = 0.0, q2 = 0.0;
+#pragma unroll
+      for (int i = 0; i < S; ++i) {
+        e += errw[i];
+        if constexpr (INIT) q2 += wsqw[i];
+      }
+      M.ws_err[(int64_t)t * tiles + tile] = e;
+      if constexpr (INIT) M.ws_wsq[tile] = q2;
     }
   };
 
@@ -439,11 +471,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     for (int t = 1; t < T; ++t) pass(std::false_type{}, std::false_type{}, t);
     pass(std::false_type{}, std::true_type{}, T);
   }
-
-  // every peer has finished writing into and reading from this CTA's buffers
-  cluster.sync();
 }
-
 // ----------------------------------------------------------------------------- amax
 __global__ void solve_amax_kernel(const __grid_constant__ SolveLaunch L, int esize) {
   const SolveMat& M = L.mats[blockIdx.y];
@@ -501,142 +529,87 @@ __global__ void finalize_kernel(const __grid_constant__ FinalizeArgs A) {
   if (lane == 0) A.mse[mat][t] = (w > 0.0) ? e / w : 0.0;
 }
 
-// Cluster size for a shape: among K >= the smallest that fits, the one with the most CTAs
-// resident at once (cluster placement inside a GPC makes some sizes pack worse), ties to the
-// smaller K; rows per CTA stay >= 32 once K exceeds the minimum. Depends on the shape and the
-// device only, so results do not depend on how many matrices share a launch.
-template <typename Kern>
-SolvePlan choose_cluster(Kern kern, const SolvePlan& base, int m, int esize, int LPB, int scb) {
-  struct Key { const void* k; int m, tiles; size_t smem; int dev; };
-  static std::mutex mu;
-  static std::vector<std::pair<Key, SolvePlan>> cache;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const Key key{reinterpret_cast<const void*>(kern), m, base.tiles, base.smem, dev};
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    for (auto& e : cache)
-      if (e.first.k == key.k && e.first.m == m && e.first.tiles == key.tiles &&
-          e.first.smem == key.smem && e.first.dev == dev)
-        return e.second;
-  }
-  SolvePlan best = base;
-  int64_t best_ctas = -1;
-  for (int K = base.K; K <= SOLVE_MAXK; ++K) {
-    const int R = (m + K - 1) / K;
-    if (K > base.K && R < 32) break;
-    const SolveSmem l = solve_smem(R, base.S, LPB, esize, scb, K, SOLVE_SEG);
-    if (l.total > 227 * 1024) continue;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)l.total) !=
-        cudaSuccess) {
-      (void)cudaGetLastError();
-      continue;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(K * base.tiles), 1, 1);
-    cfg.blockDim = dim3(SOLVE_NT, 1, 1);
-    cfg.dynamicSmemBytes = l.total;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)K;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, kern, &cfg) != cudaSuccess || active <= 0) {
-      (void)cudaGetLastError();
-      continue;
-    }
-    const int64_t ctas = (int64_t)K * std::min<int64_t>(active, base.tiles);
-    if (ctas > best_ctas) {
-      best_ctas = ctas;
-      best.K = K;
-      best.R = R;
-      best.smem = l.total;
-    }
-  }
-  std::lock_guard<std::mutex> lk(mu);
-  cache.emplace_back(key, best);
-  return best;
-}
 
 template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-cudaError_t launch_one(const SolveLaunch& L0, int count, const SolvePlan& p0, cudaStream_t st) {
-  auto kern = solve_kernel<ELEM, SCALE, SOLVE_SEG, LPB, S, F32IN>;
-  constexpr int ESZ = F32IN ? 4 : 2;
-  const SolvePlan p = choose_cluster(kern, p0, L0.m, ESZ, LPB, SCALE == SCALE_BF16 ? 2 : 1);
-  SolveLaunch L = L0;
-  L.K = p.K;
-  L.R = p.R;
+cudaError_t launch_one(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
+  auto kern = solve_kernel<ELEM, SCALE, LPB, S, F32IN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)p.smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.K * p.tiles), (unsigned)count, 1);
-  cfg.blockDim = dim3(SOLVE_NT, 1, 1);
-  cfg.dynamicSmemBytes = p.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.K;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   timing_before(st);
-  e = cudaLaunchKernelEx(&cfg, kern, L);
+  kern<<<dim3((unsigned)p.tiles, (unsigned)count, 1), SOLVE_NT, p.smem, st>>>(L);
+  e = cudaGetLastError();
   timing_after(st);
   count_launches(1);
   return e;
 }
 
-template <int ELEM, int SCALE, int LPB, int S>
+// tile width 16*S, S a power of two from LPB (one format block) to 8
+template <int ELEM, int SCALE, int LPB, bool F32IN>
+cudaError_t launch_s(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
+  switch (p.S) {
+    case 1:
+      if constexpr (LPB <= 1) return launch_one<ELEM, SCALE, LPB, 1, F32IN>(L, count, p, st);
+      break;
+    case 2:
+      if constexpr (LPB <= 2) return launch_one<ELEM, SCALE, LPB, 2, F32IN>(L, count, p, st);
+      break;
+    case 4:
+      if constexpr (LPB <= 4) return launch_one<ELEM, SCALE, LPB, 4, F32IN>(L, count, p, st);
+      break;
+    case 8: return launch_one<ELEM, SCALE, LPB, 8, F32IN>(L, count, p, st);
+    default: break;
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int ELEM, int SCALE, int LPB>
 cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const SolvePlan& p,
                          cudaStream_t st) {
-  return esize == 4 ? launch_one<ELEM, SCALE, LPB, S, true>(L, count, p, st)
-                    : launch_one<ELEM, SCALE, LPB, S, false>(L, count, p, st);
+  return esize == 4 ? launch_s<ELEM, SCALE, LPB, true>(L, count, p, st)
+                    : launch_s<ELEM, SCALE, LPB, false>(L, count, p, st);
 }
 
 }  // namespace
 
+// Tile width: the narrowest tile of whole format blocks (16*S columns, S a power of two
+// <= 8, S | n/16) that gives every thread at least 16 rows per pass, so the two barriers of
+// a pass stay a small share of it. Resident rows: as many whole sweeps (512/S rows) as fit
+// in shared memory next to the scale codes of all m rows and the reduction buffers. Depends
+// on the shape, format and input type only.
 bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ctas_hint,
                 SolvePlan* p) {
   (void)ctas_hint;
   const int B = fmt_block(kind, group);
-  if (B == 0 || m <= 0 || n <= 0 || n % B) return false;
-  const int LPB = B / SOLVE_SEG;
-  // the tile is one format block wide (NVFP4: 16, MX: 32, INT4: the group)
-  const int S = LPB;
+  if (B == 0 || m <= 0 || n <= 0 || n % B || m > (1 << 24)) return false;
+  const int LPB = B / 16;
   const int scb = kind == 0 ? 2 : 1;
-  // smallest cluster whose CTAs fit two per SM (the register limit), else one
-  const size_t budgets[2] = {SOLVE_SMEM_2PERSM, SOLVE_SMEM_1PERSM};
-  for (size_t budget : budgets) {
-    for (int K = 1; K <= SOLVE_MAXK; ++K) {
-      const int R = (int)((m + K - 1) / K);
-      const SolveSmem l = solve_smem(R, S, LPB, esize, scb, K, SOLVE_SEG);
-      if (l.total <= budget) {
-        p->S = S;
-        p->K = K;
-        p->R = R;
-        p->tiles = (int)(n / (SOLVE_SEG * S));
-        p->smem = l.total;
-        return true;
-      }
-    }
-  }
-  return false;
+  int S = LPB;
+  while (S < 8 && m * S < (int64_t)16 * SOLVE_NT && n % (32 * S) == 0) S *= 2;
+  const int NG = SOLVE_NT / S;
+  const SolveSmem base = solve_smem((int)m, 0, S, LPB, esize, scb);
+  if (base.total + 128 > SOLVE_SMEM_MAX) return false;
+  const int64_t row_bytes = (int64_t)16 * S * esize;
+  int64_t R = (int64_t)(SOLVE_SMEM_MAX - base.total - 128) / row_bytes / NG * NG;
+  R = std::min<int64_t>(R, (m + NG - 1) / NG * NG);
+  const SolveSmem l = solve_smem((int)m, (int)R, S, LPB, esize, scb);
+  if (l.total > SOLVE_SMEM_MAX) return false;
+  p->S = S;
+  p->R = (int)R;
+  p->tiles = (int)(n / (16 * S));
+  p->smem = l.total;
+  return true;
 }
 
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s) {
   switch (kind) {
     case 0:
-      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4, 4>(L, count, esize, p, s);
-      return launch_dtype<ELEM_INT4, SCALE_BF16, 8, 8>(L, count, esize, p, s);
-    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
-    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, 2>(L, count, esize, p, s);
-    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, 1>(L, count, esize, p, s);
+      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4>(L, count, esize, p, s);
+      return launch_dtype<ELEM_INT4, SCALE_BF16, 8>(L, count, esize, p, s);
+    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2>(L, count, esize, p, s);
+    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2>(L, count, esize, p, s);
+    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1>(L, count, esize, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
