@@ -71,6 +71,22 @@ __device__ __forceinline__ uint32_t quant2(float2 x, float2& q) {
   }
 }
 
+// Quantized values of a pair only (no code): E2M1 encode and decode in one step, the code
+// never leaves the conversion unit's 8-bit register.
+template <int ELEM>
+__device__ __forceinline__ float2 quant2_value(float2 x) {
+  if constexpr (ELEM == ELEM_E2M1) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h2) : "f"(x.x), "f"(x.y));
+    __half2 hv = *reinterpret_cast<__half2*>(&h2);
+    return __half22float2(hv);
+  } else {
+    return make_float2(int4_round(x.x), int4_round(x.y));
+  }
+}
+
 // ------------------------------------------------------------------ E4M3 (FN)
 // Nearest E4M3 code of u >= 0 (RNE, saturating at 448); code 0 for u that rounds to 0.
 __device__ __forceinline__ uint32_t e4m3_encode(float u) {
@@ -174,8 +190,12 @@ __device__ __forceinline__ ScaleVal project_scale_ls(float num, float den, float
   } else if constexpr (SCALE == SCALE_E8M0) {
     code = e8m0_encode(__fdividef(num, den));
   } else {
+    // num >= +0 (every w*q >= 0: q has the sign of w) and den > 0, so u >= +0; the high
+    // half of the conversion is the code of +0, so the low byte is the whole result
     const float u = __fdividef(num, __fmul_rn(den, s_t));
-    code = max(e4m3_encode(u > 0.0f ? u : 0.0f), 1u);
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(u));
+    code = max((uint32_t)out, 1u);
   }
   return scale_decode<SCALE>(code, tbl);
 }

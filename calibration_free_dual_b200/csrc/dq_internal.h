@@ -43,7 +43,8 @@ struct SolvePlan {
 };
 
 // Shared-memory carve-up of a solve CTA (same arithmetic on host and device): the resident
-// rows of W, the scale code of every (row, block) of the tile, the E4M3 table, c and 1/c,
+// rows of W (R, a whole number of sweeps), the scale code of every (row, block) of the tile
+// with the rows rounded up to whole sweeps, the E4M3 table, c and 1/c,
 // the per-warp column partials and the per-column fp64 sums (N, D, ||W_j||^2, error).
 struct SolveSmem {
   size_t w, codes, tbl, cvec, icvec, red, cols, total;
@@ -53,11 +54,12 @@ __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a -
 
 __host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, int esize,
                                                  int scb) {
-  const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32;
+  const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32, NG = SOLVE_NT / S;
+  const size_t mpad = ((size_t)m + NG - 1) / NG * NG;    // rows rounded up to whole sweeps
   SolveSmem l;
   size_t off = 0;
   l.w = off;      off = align_up(off + (size_t)R * TN * esize, 128);
-  l.codes = off;  off = align_up(off + (size_t)m * NBLK * scb, 16);
+  l.codes = off;  off = align_up(off + mpad * NBLK * scb, 16);
   l.tbl = off;    off = align_up(off + 128 * 8, 16);
   l.cvec = off;   off = align_up(off + TN * 4, 16);
   l.icvec = off;  off = align_up(off + TN * 4, 16);

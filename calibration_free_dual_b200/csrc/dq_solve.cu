@@ -64,19 +64,6 @@ __device__ __forceinline__ void zero(Raw<ESZ>& r) {
   for (int i = 0; i < ESZ * 4; ++i) r.u[i] = 0u;
 }
 
-template <int ESZ>
-__device__ __forceinline__ void load_smem(const unsigned char* Wsm, int P, Raw<ESZ>& r) {
-  const uint4* base = reinterpret_cast<const uint4*>(Wsm);
-#pragma unroll
-  for (int h = 0; h < ESZ; ++h) {
-    const uint4 v = base[chunk_pos<ESZ>(P, h)];
-    r.u[4 * h + 0] = v.x;
-    r.u[4 * h + 1] = v.y;
-    r.u[4 * h + 2] = v.z;
-    r.u[4 * h + 3] = v.w;
-  }
-}
-
 // 32 bytes from L2, not allocated in L1, kept in L2 ahead of normal lines (evict-last):
 // these rows are read again on every pass.
 __device__ __forceinline__ void ldg256_keep(const void* p, uint32_t* d) {
@@ -173,13 +160,17 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   double* errw = reinterpret_cast<double*>(smem + lay.cols);   // [S] per-warp error sums
   double* wsqw = errw + 8;                                     // [S] per-warp ||W||^2 sums
 
-  auto code_at = [&](int row) -> uint32_t {
-    if constexpr (SCB == 2) return reinterpret_cast<uint16_t*>(codes_v)[row * NBLK + bl];
-    else return reinterpret_cast<uint8_t*>(codes_v)[row * NBLK + bl];
+  // Sweep k gives this thread row g + k*NG; with NG*S = NT its piece is number tid + NT*k of
+  // the row-major tile and its block's scale code is number tid/LPB + k*NT/LPB.
+  const int code0 = tid / LPB;
+  auto code_at = [&](int k) -> uint32_t {
+    if constexpr (SCB == 2) return reinterpret_cast<uint16_t*>(codes_v)[code0 + k * (NT / LPB)];
+    else return reinterpret_cast<uint8_t*>(codes_v)[code0 + k * (NT / LPB)];
   };
-  auto set_code = [&](int row, uint32_t code) {
-    if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(codes_v)[row * NBLK + bl] = (uint16_t)code;
-    else reinterpret_cast<uint8_t*>(codes_v)[row * NBLK + bl] = (uint8_t)code;
+  auto set_code = [&](int k, uint32_t code) {
+    if constexpr (SCB == 2)
+      reinterpret_cast<uint16_t*>(codes_v)[code0 + k * (NT / LPB)] = (uint16_t)code;
+    else reinterpret_cast<uint8_t*>(codes_v)[code0 + k * (NT / LPB)] = (uint8_t)code;
   };
 
   // ---- tensor scale (NVFP4) and the code -> (r, 1/r) table
@@ -208,17 +199,18 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     icvec[tid] = __frcp_rn(cj);
   }
 
-  // ---- rows [0, min(R, m)) into shared memory (their only read from HBM)
+  // ---- rows [0, R) into shared memory (their only read from HBM); rows past m (only in the
+  // last sweep) are zeros, which add nothing to any sum
   {
     constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
-    const int rows = min(L.R, m);
     const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
     uint4* dst = reinterpret_cast<uint4*>(Wsm);
     bool bad = false;
 #pragma unroll 4
-    for (int ch = tid; ch < rows * CH; ch += NT) {
+    for (int ch = tid; ch < L.R * CH; ch += NT) {
       const int row = ch / CH, part = ch % CH;
-      const uint4 v = ldg_stream(base + (int64_t)row * pitch + part * 16);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (row < m) v = ldg_stream(base + (int64_t)row * pitch + part * 16);
       if constexpr (ESZ == 2) {
         bad |= bf16x2_nonfinite(v.x) | bf16x2_nonfinite(v.y) | bf16x2_nonfinite(v.z) |
                bf16x2_nonfinite(v.w);
@@ -251,12 +243,27 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   const int KS = min(L.R / NG, RPT);       // sweeps served from shared memory
   const int nh = n >> 1;
 
-  // row piece of sweep k: shared memory, L2, or zeros past the last row
+  // row piece of sweep k: shared memory (chunk h of piece tid + NT*k sits at
+  // ESZ*(tid + NT*k) + (h ^ sw)), else L2, or zeros past the last row
+  const uint4* smp = reinterpret_cast<const uint4*>(Wsm) + ESZ * tid;
+  const int sw = (ESZ == 2) ? ((tid >> 2) & 1) : ((tid >> 1) & 3);
+  const char* gp = gW + (int64_t)g * pitch;
+  const int64_t gstep = (int64_t)NG * pitch;
   auto fetch = [&](int k, Raw<ESZ>& dst) {
-    const int row = g + k * NG;
-    if (row >= m) zero<ESZ>(dst);
-    else if (k < KS) load_smem<ESZ>(Wsm, row * S + s, dst);
-    else load_global<ESZ>(gW + (int64_t)row * pitch, wide, dst);
+    if (k < KS) {
+#pragma unroll
+      for (int h = 0; h < ESZ; ++h) {
+        const uint4 v = smp[ESZ * NT * k + (h ^ sw)];
+        dst.u[4 * h + 0] = v.x;
+        dst.u[4 * h + 1] = v.y;
+        dst.u[4 * h + 2] = v.z;
+        dst.u[4 * h + 3] = v.w;
+      }
+    } else if (g + k * NG < m) {
+      load_global<ESZ>(gp + k * gstep, wide, dst);
+    } else {
+      zero<ESZ>(dst);
+    }
   };
 
   // per-column totals of the 32-value vectors (a: 16 columns, b: 16 columns) of all
@@ -306,20 +313,23 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     }
     bool bad = false;
 
+    // the next row's piece and (after iteration 0) its scale are fetched one row ahead
     Raw<ESZ> buf;
     fetch(0, buf);
+    ScaleVal scn;
+    if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
     for (int k = 0; k < RPT; ++k) {
       const int row = g + k * NG;
-      const bool valid = row < m;
       float2 w[8];
       unpack<ESZ>(buf, w);
-      if (k + 1 < RPT) fetch(k + 1, buf);
+      ScaleVal sc;
+      if constexpr (!INIT) sc = scn;
+      if (k + 1 < RPT) {
+        fetch(k + 1, buf);
+        if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+      }
       if constexpr (INIT) {
         if (k >= KS) bad |= nonfinite8(w);
-      }
-
-      ScaleVal sc;
-      if constexpr (INIT) {
         float a = 0.0f;
 #pragma unroll
         for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
@@ -327,14 +337,11 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
         float v;
         if (M.r0 != nullptr) {
-          v = valid ? M.r0[(int64_t)row * nb + col0 / B + bl] : 1.0f;
+          v = (row < m) ? M.r0[(int64_t)row * nb + col0 / B + bl] : 1.0f;
         } else {
           v = (a > 0.0f) ? __fdiv_rn(a, QMAX) : 1.0f;
         }
         sc = project_scale<SCALE>(v, s_t, tbl);
-      } else {
-        sc = scale_decode<SCALE>(valid ? code_at(row) : (SCALE == SCALE_BF16 ? 0x3F80u : 127u),
-                                 tbl);
       }
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
@@ -343,8 +350,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
-        const uint32_t cb = quant2<ELEM>(mul2(mul2(w[p], ic[p]), irr), q[p]);
-        if constexpr (EMIT) codes[p >> 2] |= cb << (8 * (p & 3));
+        const float2 x = mul2(mul2(w[p], ic[p]), irr);
+        if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
+        else q[p] = quant2_value<ELEM>(x);
       }
 
       if constexpr (!INIT) {
@@ -385,7 +393,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
           if (den > 0.0f) sc = project_scale_ls<SCALE>(num, den, s_t, tbl);
         }
       }
-      if (valid && lib == 0) set_code(row, sc.code);
+      if (lib == 0) set_code(k, sc.code);
 
       // c-step partial sums with the new r
       const float2 rr = make_float2(sc.r, sc.r);
@@ -398,7 +406,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
 
       if constexpr (EMIT) {
-        if (valid) {
+        if (row < m) {
           uint8_t* qp = M.q_packed + (int64_t)row * nh + (col0 + s * 16) / 2;
           *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
           if (lib == 0) {
