@@ -481,32 +481,47 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   }
 }
 // ----------------------------------------------------------------------------- amax
-__global__ void solve_amax_kernel(const __grid_constant__ SolveLaunch L, int esize) {
-  const SolveMat& M = L.mats[blockIdx.y];
-  const int64_t rows = L.m, n = L.n, ldw = M.ldw;
-  const int64_t cpr = n * esize / 16;                 // 16-byte chunks per row
-  const int64_t total = rows * cpr;
-  const char* base = reinterpret_cast<const char*>(M.W);
-  float a = 0.0f;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / cpr, part = i % cpr;
-    const uint4 v = ldg_stream(base + row * ldw * esize + part * 16);
-    if (esize == 2) {
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = bf16x2_to_f2(u[k]);
-        a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
-      }
-    } else {
-      a = fmaxf(a, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
-                         fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
-    }
+// max |W| of every matrix (NVFP4 tensor scale): one warp per row, four 16-byte loads in
+// flight per lane, maximum over the magnitude bits (for non-negative floats the bit patterns
+// order like the values; a NaN counts as larger than any number, and the solve reports it).
+template <int ESZ>
+__device__ __forceinline__ uint32_t fold_abs(uint32_t mx, const uint4& v) {
+  if constexpr (ESZ == 2) {
+    mx = __vmaxu2(mx, v.x & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.y & 0x7FFF7FFFu);
+    mx = __vmaxu2(mx, v.z & 0x7FFF7FFFu);
+    return __vmaxu2(mx, v.w & 0x7FFF7FFFu);
+  } else {
+    mx = max(mx, v.x & 0x7FFFFFFFu);
+    mx = max(mx, v.y & 0x7FFFFFFFu);
+    mx = max(mx, v.z & 0x7FFFFFFFu);
+    return max(mx, v.w & 0x7FFFFFFFu);
   }
+}
+
+template <int ESZ>
+__global__ void __launch_bounds__(256) solve_amax_kernel(const __grid_constant__ SolveLaunch L) {
+  const SolveMat& M = L.mats[blockIdx.y];
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  const int cpr = L.n * ESZ / 16;                    // 16-byte chunks per row
+  uint32_t mx = 0u;
+  for (int row = wid; row < L.m; row += nw) {
+    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(M.W) +
+                                                    (int64_t)row * M.ldw * ESZ);
+    int c = lane;
+    for (; c + 96 < cpr; c += 128) {
+      const uint4 v0 = ldg_stream(p + c), v1 = ldg_stream(p + c + 32);
+      const uint4 v2 = ldg_stream(p + c + 64), v3 = ldg_stream(p + c + 96);
+      mx = fold_abs<ESZ>(fold_abs<ESZ>(fold_abs<ESZ>(fold_abs<ESZ>(mx, v0), v1), v2), v3);
+    }
+    for (; c < cpr; c += 32) mx = fold_abs<ESZ>(mx, ldg_stream(p + c));
+  }
+  if constexpr (ESZ == 2) mx = max(mx & 0xFFFFu, mx >> 16) << 16;
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
-  if ((threadIdx.x & 31) == 0 && a > 0.0f) atomicMax(M.amax_bits, __float_as_uint(a));
+  for (int off = 16; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, off));
+  if (lane == 0 && mx != 0u) atomicMax(M.amax_bits, mx);
 }
 
 // ------------------------------------------------------------------------- finalize
@@ -623,10 +638,11 @@ cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, i
 }
 
 cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s) {
-  const int64_t chunks = (int64_t)L.m * L.n * esize / 16;
-  int blocks = (int)std::min<int64_t>((chunks + 255) / 256, 1184);
-  if (blocks < 1) blocks = 1;
-  solve_amax_kernel<<<dim3(blocks, count), 256, 0, s>>>(L, esize);
+  // about 64 warps per SM over the whole launch, at most one warp per row
+  const int warps = std::max(1, std::min(L.m, 148 * 64 / std::max(count, 1)));
+  const int blocks = (warps + 7) / 8;
+  if (esize == 4) solve_amax_kernel<4><<<dim3(blocks, count), 256, 0, s>>>(L);
+  else solve_amax_kernel<2><<<dim3(blocks, count), 256, 0, s>>>(L);
   count_launches(1);
   return cudaGetLastError();
 }
