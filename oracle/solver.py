@@ -13,6 +13,11 @@ Model: W_hat[i, j] = r[i, j // B] * q[i, j] * c[j]. One iteration runs, in this 
   r-step  r = Pi_S( fl32( sum_b W q c / sum_b (q c)^2 ) )       (kept where the sum is 0)
   c-step  c = fl32( sum_i W q r / sum_i (q r)^2 )               (kept where the sum is 0)
 Sums and the traces are binary64; the code decisions are taken on binary32 values.
+
+Ablation modes (the ai4snews summary, paragraph 2: turning on only the row scales or only
+the column scales): update="row" runs the Q- and r-steps only (c stays at its initial value),
+update="col" the Q- and c-steps only (r stays at its initial projected value). Each kept step
+is still an exact block minimiser, so the trace stays monotone.
 """
 from __future__ import annotations
 
@@ -114,15 +119,22 @@ def mse(W: np.ndarray, q: np.ndarray, r: np.ndarray, c: np.ndarray, B: int) -> f
     return float(np.sum(e * e)) / wsq
 
 
-def solve(W, fmt: Format, iters: int, r0=None, c0=None, amax=None, keep_history=False):
+UPDATES = ("both", "row", "col")
+
+
+def solve(W, fmt: Format, iters: int, r0=None, c0=None, amax=None, keep_history=False,
+          update: str = "both"):
     """Run the dual-scale BCD solve of one matrix.
 
     W: [m, n] array of binary32-representable values (bf16 or fp32 weights).
     r0 / c0: optional warm start (r0 is projected; c0 must be finite and positive).
     amax: NVFP4 only, overrides the matrix amax for the tensor scale.
+    update: "both" (the method), "row" (r only) or "col" (c only).
     Returns a dict with q (values), codes, r, r_codes, c, s_t, mse [T+1], qchange [T+1]
     and, with keep_history, the states (r, c) before each iteration's Q-step.
     """
+    if update not in UPDATES:
+        raise ValueError("update must be one of %s" % (UPDATES,))
     W = np.asarray(W, dtype=np.float64)
     m, n = W.shape
     B = fmt.block
@@ -148,8 +160,10 @@ def solve(W, fmt: Format, iters: int, r0=None, c0=None, amax=None, keep_history=
             history.append((r.copy(), c.copy(), r_codes.copy()))
         q_prev = q
         codes, q, _ = q_step(W, r, c, fmt)
-        r_codes, r, _, _ = r_step(W, q, c, r, r_codes, fmt, s_t)
-        c, _, _ = c_step(W, q, r, c, B)
+        if update != "col":
+            r_codes, r, _, _ = r_step(W, q, c, r, r_codes, fmt, s_t)
+        if update != "row":
+            c, _, _ = c_step(W, q, r, c, B)
         trace.append(mse(W, q, r, c, B))
         nprev = float(np.linalg.norm(q_prev))
         qchange.append(float(np.linalg.norm(q - q_prev)) / nprev if nprev > 0 else 0.0)
