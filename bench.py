@@ -43,7 +43,7 @@ OPS_PER_ELEM_INIT = 8
 HBM_BYTES_PER_ELEM_ITER = 2.125
 
 
-KERNEL_SOURCES = ("dq_solve.cu", "dq_device.cuh", "dq_internal.h")
+KERNEL_SOURCES = ("dq_solve.cu", "dq_solve_kernel.cuh", "dq_device.cuh", "dq_internal.h")
 PROFILE = os.path.join(ROOT, "profiles", "solve_kernel_8b_nvfp4_full.md")
 
 

@@ -14,6 +14,7 @@ DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4 = 0, 1, 2, 3
 DQ_F32, DQ_BF16 = 0, 1
 DQ_CODEC_INT4, DQ_CODEC_E2M1, DQ_CODEC_E4M3, DQ_CODEC_E8M0, DQ_CODEC_BF16 = 0, 1, 2, 3, 4
 DQ_NOALLOC_SCRATCH_BYTES = 4 << 20
+DQ_UPDATE_BOTH, DQ_UPDATE_ROW_ONLY, DQ_UPDATE_COL_ONLY = 0, 1, 2
 
 
 class dq_format(ctypes.Structure):
@@ -27,6 +28,10 @@ class dq_matrix(ctypes.Structure):
                 ("mse_trace", c_void_p)]
 
 
+class dq_solve_options(ctypes.Structure):
+    _fields_ = [("update", c_int32), ("qchange", ctypes.POINTER(c_void_p))]
+
+
 # name -> (restype, argtypes); the same names as the C ABI
 SIGNATURES = {
     "dq_status_string": (ctypes.c_char_p, [c_int32]),
@@ -35,6 +40,12 @@ SIGNATURES = {
                                             ctypes.POINTER(c_int64), dq_format, c_int32]),
     "dq_solve_batched": (c_int32, [ctypes.POINTER(dq_matrix), c_int64, c_int32, dq_format,
                                    c_int32, c_void_p, c_size_t, c_void_p]),
+    "dq_solve_workspace_bytes_ex": (c_size_t, [c_int64, ctypes.POINTER(c_int64),
+                                               ctypes.POINTER(c_int64), dq_format, c_int32,
+                                               ctypes.POINTER(dq_solve_options)]),
+    "dq_solve_batched_ex": (c_int32, [ctypes.POINTER(dq_matrix), c_int64, c_int32, dq_format,
+                                      c_int32, ctypes.POINTER(dq_solve_options), c_void_p,
+                                      c_size_t, c_void_p]),
     "dq_solve": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, dq_format, c_int32,
                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                            c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),

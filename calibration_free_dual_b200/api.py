@@ -86,9 +86,17 @@ def solve_outputs(m: int, n: int, fmt, iters: int, device) -> dict:
     )
 
 
+UPDATES = {"both": _lib.DQ_UPDATE_BOTH, "row": _lib.DQ_UPDATE_ROW_ONLY,
+           "col": _lib.DQ_UPDATE_COL_ONLY}
+
+
 def solve_batched(Ws: Iterable[torch.Tensor], fmt, iters: int, r0s=None, c0s=None,
-                  stream=None, outs=None, workspace: torch.Tensor | None = None) -> list:
-    """dq_solve_batched over a list of 2-D CUDA matrices (all bf16 or all fp32)."""
+                  stream=None, outs=None, workspace: torch.Tensor | None = None,
+                  update: str = "both", qchange: bool = False) -> list:
+    """dq_solve_batched over a list of 2-D CUDA matrices (all bf16 or all fp32).
+
+    update: "both", "row" (r only) or "col" (c only); qchange: also return the Q-change
+    trace ("qchange", [iters+1] fp64). Either option goes through dq_solve_batched_ex."""
     Ws = list(Ws)
     if not Ws:
         return []
@@ -117,13 +125,30 @@ def solve_batched(Ws: Iterable[torch.Tensor], fmt, iters: int, r0s=None, c0s=Non
             o["q_packed"].data_ptr(), o["r"].data_ptr(), o["c"].data_ptr(),
             o["block_scales"].data_ptr(), o["tensor_scale"].data_ptr(), o["mse"].data_ptr())
     lib = _lib.get()
-    need = lib.dq_solve_workspace_bytes(count, ms, ns, f, iters)
+    if update not in UPDATES:
+        raise ValueError("update must be one of %s" % sorted(UPDATES))
+    opts = None
+    if update != "both" or qchange:
+        qptrs = None
+        if qchange:
+            for o in results:
+                o["qchange"] = torch.empty((iters + 1,), dtype=torch.float64,
+                                           device=Ws[0].device)
+            qptrs = (ctypes.c_void_p * count)(*[o["qchange"].data_ptr() for o in results])
+        opts = _lib.dq_solve_options(UPDATES[update], qptrs)
+    need = lib.dq_solve_workspace_bytes_ex(count, ms, ns, f, iters,
+                                           ctypes.byref(opts) if opts is not None else None)
     if need == 0:
         raise DQError(_lib.DQ_ERR_UNSUPPORTED, "no workspace size for these shapes")
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=Ws[0].device)
-    _check(lib.dq_solve_batched(mats, count, dt, f, iters, _p(workspace), need,
-                                _stream_ptr(stream)), "dq_solve_batched")
+    if opts is None:
+        _check(lib.dq_solve_batched(mats, count, dt, f, iters, _p(workspace), need,
+                                    _stream_ptr(stream)), "dq_solve_batched")
+    else:
+        _check(lib.dq_solve_batched_ex(mats, count, dt, f, iters, ctypes.byref(opts),
+                                       _p(workspace), need, _stream_ptr(stream)),
+               "dq_solve_batched_ex")
     for o in results:
         o["_workspace"] = workspace
     return results

@@ -39,9 +39,11 @@ int dtype_size(int32_t dt) { return dt == DQ_F32 ? 4 : (dt == DQ_BF16 ? 2 : 0); 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-size_t per_matrix_ws(int tiles, int iters) {
-  // ||W||^2 partials [tiles], error partials [(iters+1) * tiles]
-  return dq::align_up(sizeof(double) * (size_t)tiles * (size_t)(iters + 2), 256);
+size_t per_matrix_ws(int tiles, int iters, bool qch) {
+  // ||W||^2 partials [tiles], error partials [(iters+1) * tiles], and with the Q-change
+  // trace its partials [(iters+1) * tiles * 2]
+  const size_t per = (size_t)(iters + 2) + (qch ? 2 * (size_t)(iters + 1) : 0);
+  return dq::align_up(sizeof(double) * (size_t)tiles * per, 256);
 }
 
 // head of the workspace: one amax word per matrix (cleared by a single memset)
@@ -100,33 +102,48 @@ int64_t dq_solve_max_rows(int64_t n, dq_format fmt, int32_t dtype) {
   while (lo < hi) {
     const int64_t mid = (lo + hi + 1) / 2;
     dq::SolvePlan p;
-    if (dq::plan_solve(mid, n, fmt.kind, fmt.group, dtype_size(dtype), 1 << 20, &p)) lo = mid;
+    if (dq::plan_solve(mid, n, fmt.kind, fmt.group, dtype_size(dtype), false, &p)) lo = mid;
     else hi = mid - 1;
   }
   return lo;
 }
 
-size_t dq_solve_workspace_bytes(int64_t count, const int64_t* m, const int64_t* n,
-                                dq_format fmt, int32_t iters) {
+size_t dq_solve_workspace_bytes_ex(int64_t count, const int64_t* m, const int64_t* n,
+                                   dq_format fmt, int32_t iters,
+                                   const dq_solve_options* options) {
   if (count <= 0 || m == nullptr || n == nullptr || iters < 0) return 0;
   if (check_format(fmt) != DQ_OK) return 0;
+  const bool qch = options != nullptr && options->qchange != nullptr;
   size_t total = amax_head(count);
   for (int64_t i = 0; i < count; ++i) {
     dq::SolvePlan p;
     // a shape is supported if some input dtype fits
-    if (!dq::plan_solve(m[i], n[i], fmt.kind, fmt.group, 2, 1 << 20, &p) &&
-        !dq::plan_solve(m[i], n[i], fmt.kind, fmt.group, 4, 1 << 20, &p))
+    if (!dq::plan_solve(m[i], n[i], fmt.kind, fmt.group, 2, qch, &p) &&
+        !dq::plan_solve(m[i], n[i], fmt.kind, fmt.group, 4, qch, &p))
       return 0;
     // room for one tile per format block, the most tiles any plan uses
-    total += per_matrix_ws((int)(n[i] / dq::fmt_block(fmt.kind, fmt.group)), iters);
+    total += per_matrix_ws((int)(n[i] / dq::fmt_block(fmt.kind, fmt.group)), iters, qch);
   }
   return total;
 }
 
-dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, dq_format fmt,
-                           int32_t iters, void* workspace, size_t workspace_bytes,
-                           void* stream) {
+size_t dq_solve_workspace_bytes(int64_t count, const int64_t* m, const int64_t* n,
+                                dq_format fmt, int32_t iters) {
+  return dq_solve_workspace_bytes_ex(count, m, n, fmt, iters, nullptr);
+}
+
+dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtype,
+                              dq_format fmt, int32_t iters, const dq_solve_options* options,
+                              void* workspace, size_t workspace_bytes, void* stream) {
   if (mats == nullptr || count <= 0 || iters < 0 || iters > (1 << 20)) return DQ_ERR_INVALID_ARG;
+  const int32_t update = options != nullptr ? options->update : DQ_UPDATE_BOTH;
+  if (update != DQ_UPDATE_BOTH && update != DQ_UPDATE_ROW_ONLY && update != DQ_UPDATE_COL_ONLY)
+    return DQ_ERR_INVALID_ARG;
+  double* const* qchange = options != nullptr ? options->qchange : nullptr;
+  const bool qch = qchange != nullptr;
+  if (qch)
+    for (int64_t i = 0; i < count; ++i)
+      if (qchange[i] == nullptr) return DQ_ERR_INVALID_ARG;
   dq_status st = check_format(fmt);
   if (st != DQ_OK) return st;
   const int esize = dtype_size(dtype);
@@ -147,7 +164,8 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
     ms[i] = d.m;
     ns[i] = d.n;
   }
-  const size_t need = dq_solve_workspace_bytes(count, ms.data(), ns.data(), fmt, iters);
+  const size_t need = dq_solve_workspace_bytes_ex(count, ms.data(), ns.data(), fmt, iters,
+                                                  options);
   if (need == 0) return DQ_ERR_UNSUPPORTED;
   if (workspace == nullptr || workspace_bytes < need) return DQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return DQ_ERR_INVALID_ARG;
@@ -162,6 +180,7 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
     unsigned* amax;
     double* wsq;
     double* err;
+    double* qch;
   };
   std::vector<Slot> slots(count);
   char* ws = static_cast<char*>(workspace);
@@ -174,13 +193,14 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
     Slot& sl = slots[i];
     // the plan depends on the matrix shape only, so a matrix gets bit-identical results
     // whether it is solved alone or inside a layer set
-    if (!dq::plan_solve(ms[i], ns[i], fmt.kind, fmt.group, esize, 1, &sl.plan))
+    if (!dq::plan_solve(ms[i], ns[i], fmt.kind, fmt.group, esize, qch, &sl.plan))
       return DQ_ERR_UNSUPPORTED;
     const int tiles_max = (int)(ns[i] / B);
     sl.amax = reinterpret_cast<unsigned*>(ws) + i;
     sl.wsq = reinterpret_cast<double*>(ws + off);
     sl.err = sl.wsq + sl.plan.tiles;
-    off += per_matrix_ws(tiles_max, iters);
+    sl.qch = qch ? sl.err + (size_t)(iters + 1) * sl.plan.tiles : nullptr;
+    off += per_matrix_ws(tiles_max, iters, qch);
   }
 
   // group by shape (order of first appearance), launch in chunks of SOLVE_MAXMATS
@@ -205,6 +225,8 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
       L.tiles = plan.tiles;
       L.count = c;
       L.wide = 1;
+      L.upd_r = update != DQ_UPDATE_COL_ONLY;
+      L.upd_c = update != DQ_UPDATE_ROW_ONLY;
       L.err_word = errp;
       for (int k = 0; k < c; ++k) {
         const int64_t idx = grp[base + k];
@@ -223,25 +245,37 @@ dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, 
         sm.tensor_scale = d.tensor_scale;
         sm.ws_err = slots[idx].err;
         sm.ws_wsq = slots[idx].wsq;
+        sm.ws_qch = slots[idx].qch;
         sm.amax_bits = slots[idx].amax;
       }
       if (fmt.kind == DQ_NVFP4) {
         if ((st = from_cuda(dq::launch_solve_amax(L, c, esize, s))) != DQ_OK) return st;
       }
-      if ((st = from_cuda(dq::launch_solve(L, c, fmt.kind, fmt.group, esize, plan, s))) != DQ_OK)
-        return st;
+      const cudaError_t e =
+          qch ? dq::launch_solve_qch(L, c, fmt.kind, fmt.group, esize, plan, s)
+              : dq::launch_solve(L, c, fmt.kind, fmt.group, esize, plan, s);
+      if ((st = from_cuda(e)) != DQ_OK) return st;
     }
   }
-  std::vector<double*> mse(count), err(count), wsq(count);
+  std::vector<double*> mse(count), err(count), wsq(count), wqch(count);
   std::vector<int> tiles(count);
   for (int64_t i = 0; i < count; ++i) {
     mse[i] = mats[i].mse_trace;
     err[i] = slots[i].err;
     wsq[i] = slots[i].wsq;
+    wqch[i] = slots[i].qch;
     tiles[i] = slots[i].plan.tiles;
   }
-  return from_cuda(dq::launch_finalize(mse.data(), err.data(), wsq.data(), tiles.data(),
+  return from_cuda(dq::launch_finalize(mse.data(), err.data(), wsq.data(), qchange,
+                                       qch ? wqch.data() : nullptr, tiles.data(),
                                        (int)count, iters, s));
+}
+
+dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype, dq_format fmt,
+                           int32_t iters, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return dq_solve_batched_ex(mats, count, dtype, fmt, iters, nullptr, workspace,
+                             workspace_bytes, stream);
 }
 
 dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, int64_t ldw,

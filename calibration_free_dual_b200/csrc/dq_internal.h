@@ -23,6 +23,7 @@ struct SolveMat {
   float* tensor_scale;
   double* ws_err;              // [(T+1) * tiles] per-iteration partial errors
   double* ws_wsq;              // [tiles] partial ||W||^2
+  double* ws_qch;              // [(T+1) * tiles * 2] Q-change partials (sum dq^2, sum q^2)
   unsigned* amax_bits;         // NVFP4: amax |W| as float bits (zeroed before the pre-pass)
 };
 
@@ -31,6 +32,7 @@ struct SolveLaunch {
   int R;                       // rows of each column tile kept in shared memory
   int tiles, count;
   int wide;                    // every W base and row pitch 32-byte aligned (256-bit loads)
+  int upd_r, upd_c;            // which scales the iterations update (both, r only, c only)
   unsigned* err_word;
   SolveMat mats[SOLVE_MAXMATS];
 };
@@ -45,15 +47,16 @@ struct SolvePlan {
 // Shared-memory carve-up of a solve CTA (same arithmetic on host and device): the resident
 // rows of W (R, a whole number of sweeps), the scale code of every (row, block) of the tile
 // with the rows rounded up to whole sweeps, the E4M3 table, c and 1/c,
-// the per-warp column partials and the per-column fp64 sums (N, D, ||W_j||^2, error).
+// the per-warp column partials and the per-warp fp64 error sums; with the Q-change trace
+// also the previous iteration's scale codes, its 1/c and per-warp Q-change sums.
 struct SolveSmem {
-  size_t w, codes, tbl, cvec, icvec, red, cols, total;
+  size_t w, codes, tbl, cvec, icvec, red, cols, pcodes, picvec, qred, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 __host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, int esize,
-                                                 int scb) {
+                                                 int scb, bool qch) {
   const int TN = 16 * S, NBLK = S / LPB, NWARP = SOLVE_NT / 32, NG = SOLVE_NT / S;
   const size_t mpad = ((size_t)m + NG - 1) / NG * NG;    // rows rounded up to whole sweeps
   SolveSmem l;
@@ -65,6 +68,9 @@ __host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, in
   l.icvec = off;  off = align_up(off + TN * 4, 16);
   l.red = off;    off = align_up(off + (size_t)NWARP * S * 32 * 4, 16);
   l.cols = off;   off = align_up(off + (size_t)4 * TN * 8, 16);
+  l.pcodes = off; if (qch) off = align_up(off + mpad * NBLK * scb, 16);
+  l.picvec = off; if (qch) off = align_up(off + TN * 4, 16);
+  l.qred = off;   if (qch) off = align_up(off + (size_t)NWARP * 2 * 8, 16);
   l.total = off;
   return l;
 }
@@ -84,13 +90,18 @@ void count_launches(int n);
 void timing_before(cudaStream_t s);
 void timing_after(cudaStream_t s);
 
-bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ctas_hint,
-                SolvePlan* p);
+// qch: the plan leaves room for the Q-change trace (its tile width, hence every result, is
+// the same either way)
+bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, SolvePlan* p);
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s);
+cudaError_t launch_solve_qch(const SolveLaunch& L, int count, int kind, int group, int esize,
+                             const SolvePlan& p, cudaStream_t s);
 cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s);
+// qchange / ws_qch may be null (no Q-change trace)
 cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* const* ws_wsq,
-                            const int* tiles, int count, int T, cudaStream_t s);
+                            double* const* qchange, double* const* ws_qch, const int* tiles,
+                            int count, int T, cudaStream_t s);
 
 struct ActLaunch {
   const void* X;

@@ -1,485 +1,10 @@
-// dq_solve.cu — dual-scale BCD solve, one column strip per CTA (sm_100a).
-//
-// Method: DualQuant ("DualQuant: Dual-scale Calibration-free Weight-and-Activation
-// Quantization for LLMs", Abstract): W ~ diag(r) Q diag(c) fitted by block coordinate
-// descent, every block updated in closed form; the quantizer is a black box and the scales
-// are projected onto the format's admissible set after each update (acceptodds.com
-// abstract of the same paper); the normalised-MSE trace of Figure 2 (b).
-//
-// B200 design. With r per (row, B-column block) and c per column, every step couples only
-// columns of one block (r-step) or rows of one column (c-step), so the solve splits exactly
-// into independent column strips. One CTA (512 threads, one per SM) owns a tile of
-// TN = 16*S columns and ALL m rows of it, so every reduction of the solve is CTA-local and
-// needs only __syncthreads:
-//   * the first R rows of the tile stay in shared memory for the whole solve (copied once
-//     from HBM); the remaining rows are read again from L2 on every pass with 256-bit loads
-//     marked evict-last (the streamed rows of all resident CTAs stay far below the 126 MB
-//     L2), the next row in flight while the current one is processed;
-//   * each thread owns one 16-column piece of a set of rows; LPB = B/16 neighbouring lanes
-//     share one format block and combine its r-step sums with xor shuffles;
-//   * Q-, r- and c-step run per row in registers with packed fp32x2 arithmetic
-//     (FMUL2/FFMA2) and the E2M1/E4M3 cvt instructions;
-//   * per pass, the per-column sums N_j, D_j go through a butterfly inside each warp (fp32)
-//     and a fixed binary64 tree across the 16 warps; the warps that own the tree also form
-//     the closed-form c_j and the pass's error terms. Two barriers per pass, no spin-waits.
-#include <algorithm>
-#include <type_traits>
-
-#include "dq_device.cuh"
-#include "dq_internal.h"
+// dq_solve.cu — host side of the solve (plan, launches), the NVFP4 amax pre-pass and the
+// trace finalisation; the solve kernel itself is in dq_solve_kernel.cuh.
+#include "dq_solve_kernel.cuh"
 
 namespace dq {
 namespace {
 
-constexpr unsigned FULL = 0xFFFFFFFFu;
-constexpr int NWARP = SOLVE_NT / 32;
-
-// 16-byte chunk position of chunk h of piece P (the 16 columns one thread owns in one row;
-// row-major [R][TN] tile, CPP chunks per piece). The 8 lanes of a quarter warp read 8
-// consecutive pieces; the swizzle spreads them over the 8 bank groups.
-template <int CPP>
-__device__ __forceinline__ int chunk_pos(int P, int h) {
-  if constexpr (CPP == 2) return 2 * P + (h ^ ((P >> 2) & 1));
-  else return 4 * P + (h ^ ((P >> 1) & 3));
-}
-
-// One row piece as raw words (bf16: 8 words; fp32: 16 words).
-template <int ESZ>
-struct Raw {
-  uint32_t u[ESZ * 4];
-};
-
-template <int ESZ>
-__device__ __forceinline__ void unpack(const Raw<ESZ>& r, float2 (&w)[8]) {
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    if constexpr (ESZ == 2) w[p] = bf16x2_to_f2(r.u[p]);
-    else w[p] = make_float2(__uint_as_float(r.u[2 * p]), __uint_as_float(r.u[2 * p + 1]));
-  }
-}
-
-template <int ESZ>
-__device__ __forceinline__ void zero(Raw<ESZ>& r) {
-#pragma unroll
-  for (int i = 0; i < ESZ * 4; ++i) r.u[i] = 0u;
-}
-
-// 32 bytes from L2, not allocated in L1, kept in L2 ahead of normal lines (evict-last):
-// these rows are read again on every pass.
-__device__ __forceinline__ void ldg256_keep(const void* p, uint32_t* d) {
-  asm volatile(
-      "ld.global.nc.L1::no_allocate.L2::evict_last.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]),
-        "=r"(d[7])
-      : "l"(p));
-}
-
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
-// A streamed row piece: 256-bit loads when every row start is 32-byte aligned, else 128-bit.
-template <int ESZ>
-__device__ __forceinline__ void load_global(const char* p, bool wide, Raw<ESZ>& r) {
-  if (wide) {
-#pragma unroll
-    for (int h = 0; h < ESZ / 2; ++h) ldg256_keep(p + 32 * h, r.u + 8 * h);
-  } else {
-#pragma unroll
-    for (int h = 0; h < ESZ; ++h) {
-      const uint4 v = ldg_stream(p + 16 * h);
-      r.u[4 * h + 0] = v.x;
-      r.u[4 * h + 1] = v.y;
-      r.u[4 * h + 2] = v.z;
-      r.u[4 * h + 3] = v.w;
-    }
-  }
-}
-
-__device__ __forceinline__ bool nonfinite8(const float2 (&w)[8]) {
-  bool bad = false;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) bad |= !isfinite(w[p].x) | !isfinite(w[p].y);
-  return bad;
-}
-
-// Butterfly reduction of 32 values over the 32/S lanes sharing piece s = lane % S.
-// Lane L ends with the S totals of indices [L - s, L - s + S) (fixed order).
-template <int S>
-__device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
-  int cnt = 32;
-#pragma unroll
-  for (int off = 16; off >= S; off >>= 1) {
-    const int half = cnt >> 1;
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i < half) {
-        const float send = upper ? v[i] : v[i + half];
-        const float keep = upper ? v[i + half] : v[i];
-        v[i] = keep + __shfl_xor_sync(FULL, send, off);
-      }
-    }
-    cnt = half;
-  }
-}
-
-// One CTA: all m rows of the column tile [tile*TN, tile*TN + TN) of matrix blockIdx.y.
-template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-__global__ void __launch_bounds__(SOLVE_NT, 1)
-solve_kernel(const __grid_constant__ SolveLaunch L) {
-  constexpr int NT = SOLVE_NT, TN = 16 * S, NBLK = S / LPB, B = 16 * LPB;
-  constexpr int NG = NT / S;             // rows covered by one sweep of all threads
-  constexpr int ESZ = F32IN ? 4 : 2;
-  constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
-  constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
-  static_assert(NBLK * LPB == S && S >= 1 && S <= 8, "tile shape");
-
-  const int m = L.m, n = L.n, T = L.T, tiles = L.tiles;
-  const int tile = blockIdx.x;
-  const SolveMat& M = L.mats[blockIdx.y];
-  const int col0 = tile * TN;
-  const int nb = n / B;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int s = tid % S, g = tid / S, bl = s / LPB, lib = s % LPB;
-  const bool wide = L.wide != 0;
-  const char* gW = reinterpret_cast<const char*>(M.W) + (int64_t)(col0 + s * 16) * ESZ;
-  const int64_t pitch = M.ldw * ESZ;
-
-  extern __shared__ __align__(128) unsigned char smem[];
-  const SolveSmem lay = solve_smem(m, L.R, S, LPB, ESZ, SCB);
-  unsigned char* Wsm = smem + lay.w;
-  void* codes_v = smem + lay.codes;
-  float2* tbl = reinterpret_cast<float2*>(smem + lay.tbl);
-  float* cvec = reinterpret_cast<float*>(smem + lay.cvec);
-  float* icvec = reinterpret_cast<float*>(smem + lay.icvec);
-  float* red = reinterpret_cast<float*>(smem + lay.red);
-  double* errw = reinterpret_cast<double*>(smem + lay.cols);   // [S] per-warp error sums
-  double* wsqw = errw + 8;                                     // [S] per-warp ||W||^2 sums
-
-  // Sweep k gives this thread row g + k*NG; with NG*S = NT its piece is number tid + NT*k of
-  // the row-major tile and its block's scale code is number tid/LPB + k*NT/LPB.
-  const int code0 = tid / LPB;
-  auto code_at = [&](int k) -> uint32_t {
-    if constexpr (SCB == 2) return reinterpret_cast<uint16_t*>(codes_v)[code0 + k * (NT / LPB)];
-    else return reinterpret_cast<uint8_t*>(codes_v)[code0 + k * (NT / LPB)];
-  };
-  auto set_code = [&](int k, uint32_t code) {
-    if constexpr (SCB == 2)
-      reinterpret_cast<uint16_t*>(codes_v)[code0 + k * (NT / LPB)] = (uint16_t)code;
-    else reinterpret_cast<uint8_t*>(codes_v)[code0 + k * (NT / LPB)] = (uint8_t)code;
-  };
-
-  // ---- tensor scale (NVFP4) and the code -> (r, 1/r) table
-  float s_t = 1.0f;
-  if constexpr (SCALE == SCALE_E4M3) {
-    s_t = nvfp4_tensor_scale(__uint_as_float(*M.amax_bits));
-    if (tid < 128) {
-      const uint32_t code = (tid == 0 || tid == 127) ? 1u : (uint32_t)tid;
-      const float r = __fmul_rn(s_t, e4m3_decode(code));
-      tbl[tid] = make_float2(r, __frcp_rn(r));
-    }
-    if (tile == 0 && tid == 0 && M.tensor_scale != nullptr) *M.tensor_scale = s_t;
-  }
-
-  // ---- column scales: c0 or 1
-  if (tid < TN) {
-    float cj = 1.0f;
-    if (M.c0 != nullptr) {
-      cj = M.c0[col0 + tid];
-      if (!(cj > 0.0f && cj <= 3.0e38f)) {
-        atomicOr(L.err_word, ERRBIT_BADWARM);
-        cj = 1.0f;
-      }
-    }
-    cvec[tid] = cj;
-    icvec[tid] = __frcp_rn(cj);
-  }
-
-  // ---- rows [0, R) into shared memory (their only read from HBM); rows past m (only in the
-  // last sweep) are zeros, which add nothing to any sum
-  {
-    constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
-    const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
-    uint4* dst = reinterpret_cast<uint4*>(Wsm);
-    bool bad = false;
-#pragma unroll 4
-    for (int ch = tid; ch < L.R * CH; ch += NT) {
-      const int row = ch / CH, part = ch % CH;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < m) v = ldg_stream(base + (int64_t)row * pitch + part * 16);
-      if constexpr (ESZ == 2) {
-        bad |= bf16x2_nonfinite(v.x) | bf16x2_nonfinite(v.y) | bf16x2_nonfinite(v.z) |
-               bf16x2_nonfinite(v.w);
-      } else {
-        bad |= ((v.x & 0x7F800000u) == 0x7F800000u) | ((v.y & 0x7F800000u) == 0x7F800000u) |
-               ((v.z & 0x7F800000u) == 0x7F800000u) | ((v.w & 0x7F800000u) == 0x7F800000u);
-      }
-      dst[chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ)] = v;
-    }
-    if (bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
-  }
-  __syncthreads();
-
-  float2 cc[8], ic[8];
-  auto load_c = [&]() {
-    const float4* cv = reinterpret_cast<const float4*>(cvec + s * 16);
-    const float4* iv = reinterpret_cast<const float4*>(icvec + s * 16);
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float4 a = cv[h], b = iv[h];
-      cc[2 * h] = make_float2(a.x, a.y);
-      cc[2 * h + 1] = make_float2(a.z, a.w);
-      ic[2 * h] = make_float2(b.x, b.y);
-      ic[2 * h + 1] = make_float2(b.z, b.w);
-    }
-  };
-  load_c();
-
-  const int RPT = (m + NG - 1) / NG;       // sweeps per pass (uniform: shuffles below)
-  const int KS = min(L.R / NG, RPT);       // sweeps served from shared memory
-  const int nh = n >> 1;
-
-  // row piece of sweep k: shared memory (chunk h of piece tid + NT*k sits at
-  // ESZ*(tid + NT*k) + (h ^ sw)), else L2, or zeros past the last row
-  const uint4* smp = reinterpret_cast<const uint4*>(Wsm) + ESZ * tid;
-  const int sw = (ESZ == 2) ? ((tid >> 2) & 1) : ((tid >> 1) & 3);
-  const char* gp = gW + (int64_t)g * pitch;
-  const int64_t gstep = (int64_t)NG * pitch;
-  auto fetch = [&](int k, Raw<ESZ>& dst) {
-    if (k < KS) {
-#pragma unroll
-      for (int h = 0; h < ESZ; ++h) {
-        const uint4 v = smp[ESZ * NT * k + (h ^ sw)];
-        dst.u[4 * h + 0] = v.x;
-        dst.u[4 * h + 1] = v.y;
-        dst.u[4 * h + 2] = v.z;
-        dst.u[4 * h + 3] = v.w;
-      }
-    } else if (g + k * NG < m) {
-      load_global<ESZ>(gp + k * gstep, wide, dst);
-    } else {
-      zero<ESZ>(dst);
-    }
-  };
-
-  // per-column totals of the 32-value vectors (a: 16 columns, b: 16 columns) of all
-  // threads; thread tid < 32*S (lane e of warp sj) returns the total of value e of piece sj
-  auto column_totals = [&](const float2 (&a)[8], const float2 (&b)[8]) -> double {
-    float v[32];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      v[2 * p] = a[p].x;
-      v[2 * p + 1] = a[p].y;
-      v[16 + 2 * p] = b[p].x;
-      v[16 + 2 * p + 1] = b[p].y;
-    }
-    transpose_reduce<S>(v, lane);
-#pragma unroll
-    for (int i = 0; i < S; ++i) red[(warp * S + s) * 32 + (lane - s) + i] = v[i];
-    __syncthreads();
-    double tot = 0.0;
-    if (tid < 32 * S) {
-      double va[NWARP];
-#pragma unroll
-      for (int wp = 0; wp < NWARP; ++wp) va[wp] = (double)red[wp * S * 32 + tid];
-#pragma unroll
-      for (int st = 1; st < NWARP; st <<= 1) {
-#pragma unroll
-        for (int i = 0; i + st < NWARP; i += 2 * st) va[i] += va[i + st];
-      }
-      tot = va[0];
-    }
-    return tot;
-  };
-
-  double Sj = 0.0;          // ||W_j||^2 of column sj*16 + lane (threads tid < 32*S, lane < 16)
-
-  // One pass over all rows of the tile. INIT: iteration 0 (scales from absmax or r0,
-  // c = c0); otherwise one BCD iteration (Q-step, r-step + projection, c-step). EMIT: the
-  // returned state is written.
-  auto pass = [&](auto init_tag, auto emit_tag, const int t) {
-    constexpr bool INIT = decltype(init_tag)::value;
-    constexpr bool EMIT = decltype(emit_tag)::value;
-    float2 accN[8], accD[8], accS[INIT ? 8 : 1];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      accN[p] = make_float2(0.f, 0.f);
-      accD[p] = make_float2(0.f, 0.f);
-      if constexpr (INIT) accS[p] = make_float2(0.f, 0.f);
-    }
-    bool bad = false;
-
-    // the next row's piece and (after iteration 0) its scale are fetched one row ahead
-    Raw<ESZ> buf;
-    fetch(0, buf);
-    ScaleVal scn;
-    if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
-    for (int k = 0; k < RPT; ++k) {
-      const int row = g + k * NG;
-      float2 w[8];
-      unpack<ESZ>(buf, w);
-      ScaleVal sc;
-      if constexpr (!INIT) sc = scn;
-      if (k + 1 < RPT) {
-        fetch(k + 1, buf);
-        if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
-      }
-      if constexpr (INIT) {
-        if (k >= KS) bad |= nonfinite8(w);
-        float a = 0.0f;
-#pragma unroll
-        for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
-#pragma unroll
-        for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
-        float v;
-        if (M.r0 != nullptr) {
-          v = (row < m) ? M.r0[(int64_t)row * nb + col0 / B + bl] : 1.0f;
-        } else {
-          v = (a > 0.0f) ? __fdiv_rn(a, QMAX) : 1.0f;
-        }
-        sc = project_scale<SCALE>(v, s_t, tbl);
-      }
-
-      // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
-      float2 q[8];
-      uint32_t codes[2] = {0u, 0u};
-      const float2 irr = make_float2(sc.ir, sc.ir);
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const float2 x = mul2(mul2(w[p], ic[p]), irr);
-        if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
-        else q[p] = quant2_value<ELEM>(x);
-      }
-
-      if constexpr (!INIT) {
-        // r-step: least squares over the block, then projection
-        if constexpr (SCALE == SCALE_BF16) {
-          // INT4's fine bf16 scale grid: block sums in binary64 keep projection decisions
-          // on the exact least-squares quotient
-          double num = 0.0, den = 0.0;
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const double qcx = (double)q[p].x * (double)cc[p].x;
-            const double qcy = (double)q[p].y * (double)cc[p].y;
-            num = fma((double)w[p].x, qcx, num);
-            num = fma((double)w[p].y, qcy, num);
-            den = fma(qcx, qcx, den);
-            den = fma(qcy, qcy, den);
-          }
-#pragma unroll
-          for (int off = 1; off < LPB; off <<= 1) {
-            num += __shfl_xor_sync(FULL, num, off);
-            den += __shfl_xor_sync(FULL, den, off);
-          }
-          if (den > 0.0) sc = project_scale<SCALE>(__double2float_rn(num / den), s_t, tbl);
-        } else {
-          float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const float2 qc = mul2(q[p], cc[p]);
-            num2 = fma2(w[p], qc, num2);
-            den2 = fma2(qc, qc, den2);
-          }
-          float num = num2.x + num2.y, den = den2.x + den2.y;
-#pragma unroll
-          for (int off = 1; off < LPB; off <<= 1) {
-            num += __shfl_xor_sync(FULL, num, off);
-            den += __shfl_xor_sync(FULL, den, off);
-          }
-          if (den > 0.0f) sc = project_scale_ls<SCALE>(num, den, s_t, tbl);
-        }
-      }
-      if (lib == 0) set_code(k, sc.code);
-
-      // c-step partial sums with the new r
-      const float2 rr = make_float2(sc.r, sc.r);
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const float2 qr = mul2(q[p], rr);
-        accN[p] = fma2(w[p], qr, accN[p]);
-        accD[p] = fma2(qr, qr, accD[p]);
-        if constexpr (INIT) accS[p] = fma2(w[p], w[p], accS[p]);
-      }
-
-      if constexpr (EMIT) {
-        if (row < m) {
-          uint8_t* qp = M.q_packed + (int64_t)row * nh + (col0 + s * 16) / 2;
-          *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
-          if (lib == 0) {
-            const int64_t bi = (int64_t)row * nb + col0 / B + bl;
-            M.r[bi] = sc.r;
-            if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(M.bscale)[bi] = (uint16_t)sc.code;
-            else reinterpret_cast<uint8_t*>(M.bscale)[bi] = (uint8_t)sc.code;
-          }
-        }
-      }
-    }
-    if (INIT && bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
-
-    // ---- column sums (iteration 0 first forms ||W_j||^2, kept by its owner thread)
-    if constexpr (INIT) {
-      float2 zero2[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) zero2[p] = make_float2(0.f, 0.f);
-      Sj = column_totals(accS, zero2);
-      __syncthreads();                       // the reduction buffer is reused
-    }
-    const double nd = column_totals(accN, accD);
-
-    // ---- c-step (closed form) and this pass's error terms: warps 0..S-1, lanes 0..15
-    if (tid < 32 * S) {
-      const double Dj = __shfl_down_sync(FULL, nd, 16);
-      double e = 0.0, q2 = 0.0;
-      if (lane < 16) {
-        const int j = warp * 16 + lane;
-        const double Nj = nd;
-        float cj = cvec[j];
-        if (!INIT && Dj > 0.0) {
-          cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
-          cvec[j] = cj;
-          icvec[j] = __frcp_rn(cj);
-        }
-        if (EMIT) M.c[col0 + j] = cj;
-        const double cd = (double)cj;
-        e = Sj - 2.0 * cd * Nj + cd * cd * Dj;
-        if constexpr (INIT) q2 = Sj;
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        e += __shfl_xor_sync(FULL, e, off);
-        if constexpr (INIT) q2 += __shfl_xor_sync(FULL, q2, off);
-      }
-      if (lane == 0) {
-        errw[warp] = e;
-        if constexpr (INIT) wsqw[warp] = q2;
-      }
-    }
-    __syncthreads();
-    if constexpr (!INIT) load_c();
-    if (tid == 0) {
-      double e = 0.0, q2 = 0.0;
-#pragma unroll
-      for (int i = 0; i < S; ++i) {
-        e += errw[i];
-        if constexpr (INIT) q2 += wsqw[i];
-      }
-      M.ws_err[(int64_t)t * tiles + tile] = e;
-      if constexpr (INIT) M.ws_wsq[tile] = q2;
-    }
-  };
-
-  if (T == 0) {
-    pass(std::true_type{}, std::true_type{}, 0);
-  } else {
-    pass(std::true_type{}, std::false_type{}, 0);
-    for (int t = 1; t < T; ++t) pass(std::false_type{}, std::false_type{}, t);
-    pass(std::false_type{}, std::true_type{}, T);
-  }
-}
 // ----------------------------------------------------------------------------- amax
 // max |W| of every matrix (NVFP4 tensor scale): one warp per row, four 16-byte loads in
 // flight per lane, maximum over the magnitude bits (for non-negative floats the bit patterns
@@ -529,6 +54,8 @@ struct FinalizeArgs {
   double* mse[SOLVE_MAXMATS];
   double* err[SOLVE_MAXMATS];
   double* wsq[SOLVE_MAXMATS];
+  double* qout[SOLVE_MAXMATS];   // null: no Q-change trace
+  double* qch[SOLVE_MAXMATS];
   int tiles[SOLVE_MAXMATS];
   int T;
 };
@@ -550,48 +77,24 @@ __global__ void finalize_kernel(const __grid_constant__ FinalizeArgs A) {
     w += __shfl_xor_sync(FULL, w, off);
   }
   if (lane == 0) A.mse[mat][t] = (w > 0.0) ? e / w : 0.0;
-}
-
-
-template <int ELEM, int SCALE, int LPB, int S, bool F32IN>
-cudaError_t launch_one(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
-  auto kern = solve_kernel<ELEM, SCALE, LPB, S, F32IN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)p.smem);
-  if (e != cudaSuccess) return e;
-  timing_before(st);
-  kern<<<dim3((unsigned)p.tiles, (unsigned)count, 1), SOLVE_NT, p.smem, st>>>(L);
-  e = cudaGetLastError();
-  timing_after(st);
-  count_launches(1);
-  return e;
-}
-
-// tile width 16*S, S a power of two from LPB (one format block) to 8
-template <int ELEM, int SCALE, int LPB, bool F32IN>
-cudaError_t launch_s(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
-  switch (p.S) {
-    case 1:
-      if constexpr (LPB <= 1) return launch_one<ELEM, SCALE, LPB, 1, F32IN>(L, count, p, st);
-      break;
-    case 2:
-      if constexpr (LPB <= 2) return launch_one<ELEM, SCALE, LPB, 2, F32IN>(L, count, p, st);
-      break;
-    case 4:
-      if constexpr (LPB <= 4) return launch_one<ELEM, SCALE, LPB, 4, F32IN>(L, count, p, st);
-      break;
-    case 8: return launch_one<ELEM, SCALE, LPB, 8, F32IN>(L, count, p, st);
-    default: break;
+  if (A.qout[mat] != nullptr) {
+    // sqrt(sum (q_t - q_{t-1})^2) / sqrt(sum q_{t-1}^2); both sums exact, so their order is free
+    double d = 0.0, p = 0.0;
+    if (t >= 2) {
+      for (int i = lane; i < tiles; i += 32) {
+        d += A.qch[mat][2 * ((int64_t)t * tiles + i)];
+        p += A.qch[mat][2 * ((int64_t)t * tiles + i) + 1];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      d += __shfl_xor_sync(FULL, d, off);
+      p += __shfl_xor_sync(FULL, p, off);
+    }
+    if (lane == 0) A.qout[mat][t] = (p > 0.0) ? sqrt(d) / sqrt(p) : 0.0;
   }
-  return cudaErrorInvalidValue;
 }
 
-template <int ELEM, int SCALE, int LPB>
-cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const SolvePlan& p,
-                         cudaStream_t st) {
-  return esize == 4 ? launch_s<ELEM, SCALE, LPB, true>(L, count, p, st)
-                    : launch_s<ELEM, SCALE, LPB, false>(L, count, p, st);
-}
 
 }  // namespace
 
@@ -599,10 +102,9 @@ cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const Solve
 // <= 8, S | n/16) that gives every thread at least 16 rows per pass, so the two barriers of
 // a pass stay a small share of it. Resident rows: as many whole sweeps (512/S rows) as fit
 // in shared memory next to the scale codes of all m rows and the reduction buffers. Depends
-// on the shape, format and input type only.
-bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ctas_hint,
-                SolvePlan* p) {
-  (void)ctas_hint;
+// on the shape, format and input type only (the Q-change trace shrinks R, which moves rows
+// between shared memory and L2 but changes no result).
+bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, SolvePlan* p) {
   const int B = fmt_block(kind, group);
   if (B == 0 || m <= 0 || n <= 0 || n % B || m > (1 << 24)) return false;
   const int LPB = B / 16;
@@ -610,12 +112,12 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ct
   int S = LPB;
   while (S < 8 && m * S < (int64_t)16 * SOLVE_NT && n % (32 * S) == 0) S *= 2;
   const int NG = SOLVE_NT / S;
-  const SolveSmem base = solve_smem((int)m, 0, S, LPB, esize, scb);
+  const SolveSmem base = solve_smem((int)m, 0, S, LPB, esize, scb, qch);
   if (base.total + 128 > SOLVE_SMEM_MAX) return false;
   const int64_t row_bytes = (int64_t)16 * S * esize;
   int64_t R = (int64_t)(SOLVE_SMEM_MAX - base.total - 128) / row_bytes / NG * NG;
   R = std::min<int64_t>(R, (m + NG - 1) / NG * NG);
-  const SolveSmem l = solve_smem((int)m, (int)R, S, LPB, esize, scb);
+  const SolveSmem l = solve_smem((int)m, (int)R, S, LPB, esize, scb, qch);
   if (l.total > SOLVE_SMEM_MAX) return false;
   p->S = S;
   p->R = (int)R;
@@ -626,15 +128,7 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, int64_t ct
 
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s) {
-  switch (kind) {
-    case 0:
-      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4>(L, count, esize, p, s);
-      return launch_dtype<ELEM_INT4, SCALE_BF16, 8>(L, count, esize, p, s);
-    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2>(L, count, esize, p, s);
-    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2>(L, count, esize, p, s);
-    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1>(L, count, esize, p, s);
-    default: return cudaErrorInvalidValue;
-  }
+  return launch_solve_formats<false>(L, count, kind, group, esize, p, s);
 }
 
 cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s) {
@@ -648,7 +142,8 @@ cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaSt
 }
 
 cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* const* ws_wsq,
-                            const int* tiles, int count, int T, cudaStream_t s) {
+                            double* const* qchange, double* const* ws_qch, const int* tiles,
+                            int count, int T, cudaStream_t s) {
   for (int base = 0; base < count; base += SOLVE_MAXMATS) {
     FinalizeArgs A = {};
     const int c = std::min(SOLVE_MAXMATS, count - base);
@@ -656,6 +151,8 @@ cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* c
       A.mse[i] = mse[base + i];
       A.err[i] = ws_err[base + i];
       A.wsq[i] = ws_wsq[base + i];
+      A.qout[i] = qchange != nullptr ? qchange[base + i] : nullptr;
+      A.qch[i] = ws_qch != nullptr ? ws_qch[base + i] : nullptr;
       A.tiles[i] = tiles[base + i];
     }
     A.T = T;

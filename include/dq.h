@@ -101,10 +101,40 @@ DQ_API size_t dq_solve_workspace_bytes(int64_t count, const int64_t* m, const in
  * (DualQuant Abstract: BCD with closed-form updates; acceptodds abstract: projection of the
  * scales after each update; Figure 2 (b): the trace, monotone by Theorem 1 (i)).
  * Returns DQ_ERR_SHAPE if some n is not a multiple of fmt.group, DQ_ERR_UNSUPPORTED if a
- * matrix has more rows than the cluster-resident kernel holds (see dq_solve_max_rows). */
+ * matrix has more rows than the kernel holds (see dq_solve_max_rows). */
 DQ_API dq_status dq_solve_batched(const dq_matrix* mats, int64_t count, int32_t dtype,
                                   dq_format fmt, int32_t iters, void* workspace,
                                   size_t workspace_bytes, void* stream);
+
+/* Which scales the iterations update: both (the method), only r (the c-step is skipped, c
+ * stays at c0 or 1) or only c (the r-step and its projection are skipped, r stays at its
+ * initial projected value). The ablation of the ai4snews summary of DualQuant, paragraph 2
+ * (turning on only the row or only the column scales). */
+typedef enum { DQ_UPDATE_BOTH = 0, DQ_UPDATE_ROW_ONLY = 1, DQ_UPDATE_COL_ONLY = 2 } dq_update;
+
+/* Options of dq_solve_batched_ex. A NULL options pointer means {DQ_UPDATE_BOTH, NULL}.
+ *   update   dq_update
+ *   qchange  NULL, or a host array of `count` device pointers, each to [iters+1] fp64 that
+ *            receive ||Q^t - Q^(t-1)||_F / ||Q^(t-1)||_F (DualQuant paper, Figure 2 (a)),
+ *            with Q^t the Q-step result of iteration t and entries 0 and 1 equal to 0. The
+ *            trace costs a second quantization of every element per iteration from t = 2
+ *            on; it changes no other output. */
+typedef struct {
+  int32_t update;
+  double* const* qchange;
+} dq_solve_options;
+
+/* Workspace for dq_solve_batched_ex with these options (the Q-change trace needs more). */
+DQ_API size_t dq_solve_workspace_bytes_ex(int64_t count, const int64_t* m, const int64_t* n,
+                                          dq_format fmt, int32_t iters,
+                                          const dq_solve_options* options);
+
+/* dq_solve_batched with options. DQ_ERR_INVALID_ARG for an unknown `update` or a null
+ * pointer inside `qchange`. */
+DQ_API dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtype,
+                                     dq_format fmt, int32_t iters,
+                                     const dq_solve_options* options, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /* Single-matrix form of dq_solve_batched (same semantics, flat arguments). */
 DQ_API dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, int64_t ldw,

@@ -101,3 +101,27 @@ def test_no_cpu_fallback(dq):
         dq.solve(torch.zeros(16, 32), "NVFP4", 2)
     with pytest.raises(TypeError):
         dq.act_quant(torch.zeros(4, 32), "NVFP4")
+
+
+def test_solve_options_validation_and_workspace(dq):
+    """dq_solve_batched_ex: an unknown update mode or a null Q-change pointer is rejected
+    before anything reaches CUDA; the Q-change trace needs more workspace."""
+    f = dq.fmt_of("MXFP4")
+    m = (ctypes.c_int64 * 1)(512)
+    n = (ctypes.c_int64 * 1)(2048)
+    plain = dq.dq_solve_workspace_bytes(1, m, n, f, 16)
+    both = dq._lib.dq_solve_options(dq.DQ_UPDATE_BOTH, None)
+    assert dq.dq_solve_workspace_bytes_ex(1, m, n, f, 16, ctypes.byref(both)) == plain
+    assert dq.dq_solve_workspace_bytes_ex(1, m, n, f, 16, None) == plain
+    qptr = (ctypes.c_void_p * 1)(0x1000)
+    traced = dq._lib.dq_solve_options(dq.DQ_UPDATE_ROW_ONLY, qptr)
+    assert dq.dq_solve_workspace_bytes_ex(1, m, n, f, 16, ctypes.byref(traced)) > plain
+    mats = (dq.dq_matrix * 1)()
+    mats[0] = dq.dq_matrix(0x1000, 512, 2048, 2048, None, None, 0x1000, 0x1000, 0x1000,
+                           0x1000, 0x1000, 0x1000)
+    bad_mode = dq._lib.dq_solve_options(5, None)
+    assert dq.dq_solve_batched_ex(mats, 1, dq.DQ_BF16, f, 16, ctypes.byref(bad_mode), None, 0,
+                                  None) == 1
+    null_trace = dq._lib.dq_solve_options(dq.DQ_UPDATE_BOTH, (ctypes.c_void_p * 1)(None))
+    assert dq.dq_solve_batched_ex(mats, 1, dq.DQ_BF16, f, 16, ctypes.byref(null_trace), None,
+                                  0, None) == 1

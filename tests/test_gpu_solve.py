@@ -1,7 +1,7 @@
 """Parity of the CUDA solve with the oracle on seeded inputs (B200).
 
-Sizes span several column tiles, multi-CTA clusters and ragged row splits while the oracle
-still finishes in seconds. Tolerances are the ones written out in tests/_parity.py.
+Sizes span several column tiles, ragged last sweeps and tiles whose lower rows are re-read
+from L2 on every pass, while the oracle still finishes in seconds. Tolerances are the ones written out in tests/_parity.py.
 """
 import numpy as np
 import pytest
@@ -72,6 +72,29 @@ def test_solve_matches_oracle(dq, fmt_name, dtype, m, n, iters):
     compare_solve(h, ora, fmt, label=f"{fmt_name}/{dtype}/{m}x{n}")
     assert_monotone(h["mse"], label=fmt_name)
     assert h["mse"][-1] <= h["mse"][0]
+
+
+@pytest.mark.parametrize("fmt_name,m,n", [("NVFP4", 3000, 256), ("MXINT4", 8000, 64),
+                                           ("INT4_G64", 2600, 128)])
+def test_l2_streamed_rows_both_load_widths(dq, fmt_name, m, n):
+    """Tall tiles keep only their top rows in shared memory and re-read the rest every pass:
+    256-bit loads when every row starts 32-byte aligned, 128-bit loads otherwise (a row
+    pitch of n + 8 bf16 elements). Both give identical results, and they match the oracle."""
+    W = _matrix(4242 + m, m, n, "bf16")
+    h = _run(dq, W, fmt_name, 8)
+    padded = torch.zeros((m, n + 8), dtype=torch.bfloat16)
+    padded[:, :n] = W
+    view = padded.cuda()[:, :n]
+    assert (view.stride(0) * 2) % 32 == 16
+    out = dq.solve(view, fmt_name, 8)
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    hp = to_host(out)
+    for key in ("q_packed", "r", "c", "block_scales", "mse"):
+        np.testing.assert_array_equal(hp[key], h[key], err_msg=key)
+    fmt = oracle_format(fmt_name)
+    ora = S.solve(W.float().numpy().astype(np.float64), fmt, 8)
+    compare_solve(h, ora, fmt, label=f"{fmt_name}/{m}x{n}/streamed")
 
 
 def test_config1_tile_full(dq):
