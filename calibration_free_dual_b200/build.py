@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdq.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["dq_api.cu", "dq_solve.cu", "dq_solve_qch.cu", "dq_act.cu", "dq_codec.cu",
+SOURCES = ["dq_api.cu", "dq_solve.cu", "dq_solve_ext.cu", "dq_act.cu", "dq_codec.cu",
            "dq_noalloc.cu"]
 HEADERS = ["dq_device.cuh", "dq_internal.h", "dq_solve_kernel.cuh"]
 

@@ -227,6 +227,7 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
       L.wide = 1;
       L.upd_r = update != DQ_UPDATE_COL_ONLY;
       L.upd_c = update != DQ_UPDATE_ROW_ONLY;
+      L.qch = qch;
       L.err_word = errp;
       for (int k = 0; k < c; ++k) {
         const int64_t idx = grp[base + k];
@@ -252,7 +253,8 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
         if ((st = from_cuda(dq::launch_solve_amax(L, c, esize, s))) != DQ_OK) return st;
       }
       const cudaError_t e =
-          qch ? dq::launch_solve_qch(L, c, fmt.kind, fmt.group, esize, plan, s)
+          (qch || update != DQ_UPDATE_BOTH)
+              ? dq::launch_solve_ext(L, c, fmt.kind, fmt.group, esize, plan, s)
               : dq::launch_solve(L, c, fmt.kind, fmt.group, esize, plan, s);
       if ((st = from_cuda(e)) != DQ_OK) return st;
     }

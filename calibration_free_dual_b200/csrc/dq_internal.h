@@ -32,7 +32,8 @@ struct SolveLaunch {
   int R;                       // rows of each column tile kept in shared memory
   int tiles, count;
   int wide;                    // every W base and row pitch 32-byte aligned (256-bit loads)
-  int upd_r, upd_c;            // which scales the iterations update (both, r only, c only)
+  int upd_r, upd_c;            // extended kernel: which scales the iterations update
+  int qch;                     // extended kernel: record the Q-change trace
   unsigned* err_word;
   SolveMat mats[SOLVE_MAXMATS];
 };
@@ -95,7 +96,8 @@ void timing_after(cudaStream_t s);
 bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, SolvePlan* p);
 cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, int esize,
                          const SolvePlan& p, cudaStream_t s);
-cudaError_t launch_solve_qch(const SolveLaunch& L, int count, int kind, int group, int esize,
+// the extended instantiation: update modes and the Q-change trace (L.upd_r, L.upd_c, L.qch)
+cudaError_t launch_solve_ext(const SolveLaunch& L, int count, int kind, int group, int esize,
                              const SolvePlan& p, cudaStream_t s);
 cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s);
 // qchange / ws_qch may be null (no Q-change trace)

@@ -130,10 +130,12 @@ __device__ __forceinline__ void transpose_reduce(float (&v)[32], int lane) {
 }
 
 // One CTA: all m rows of the column tile [tile*TN, tile*TN + TN) of matrix blockIdx.y.
-// QCH: also the Q-change trace of Figure 2 (a): from the second iteration on, every row
-// re-quantizes W with the previous iteration's (r, c), kept in shared memory, and adds
-// sum (q - q_prev)^2 and sum q_prev^2 (exact: multiples of 1/4 far below 2^24).
-template <int ELEM, int SCALE, int LPB, int S, bool F32IN, bool QCH>
+// EXT (the extended instantiation; the plain one updates both scales and records no Q-change):
+// runtime flags select which scales the iterations update, and on request the Q-change
+// trace of Figure 2 (a): from the second iteration on, every row re-quantizes W with the
+// previous iteration's (r, c), kept in shared memory, and adds sum (q - q_prev)^2 and
+// sum q_prev^2 (exact: multiples of 1/4 far below 2^24).
+template <int ELEM, int SCALE, int LPB, int S, bool F32IN, bool EXT>
 __global__ void __launch_bounds__(SOLVE_NT, 1)
 solve_kernel(const __grid_constant__ SolveLaunch L) {
   constexpr int NT = SOLVE_NT, TN = 16 * S, NBLK = S / LPB, B = 16 * LPB;
@@ -155,7 +157,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   const int64_t pitch = M.ldw * ESZ;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const SolveSmem lay = solve_smem(m, L.R, S, LPB, ESZ, SCB, QCH);
+  const bool upd_r = !EXT || L.upd_r != 0, upd_c = !EXT || L.upd_c != 0;
+  const bool qch = EXT && L.qch != 0;
+  const SolveSmem lay = solve_smem(m, L.R, S, LPB, ESZ, SCB, qch);
   unsigned char* Wsm = smem + lay.w;
   void* codes_v = smem + lay.codes;
   float2* tbl = reinterpret_cast<float2*>(smem + lay.tbl);
@@ -164,10 +168,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   float* red = reinterpret_cast<float*>(smem + lay.red);
   double* errw = reinterpret_cast<double*>(smem + lay.cols);   // [S] per-warp error sums
   double* wsqw = errw + 8;                                     // [S] per-warp ||W||^2 sums
-  void* pcodes_v = smem + lay.pcodes;                          // QCH: previous scale codes
-  float* picvec = reinterpret_cast<float*>(smem + lay.picvec); // QCH: previous 1/c
-  double* qred = reinterpret_cast<double*>(smem + lay.qred);   // QCH: per-warp sums
-  const bool upd_r = L.upd_r != 0, upd_c = L.upd_c != 0;
+  void* pcodes_v = smem + lay.pcodes;                          // Q-change: previous codes
+  float* picvec = reinterpret_cast<float*>(smem + lay.picvec); // Q-change: previous 1/c
+  double* qred = reinterpret_cast<double*>(smem + lay.qred);   // Q-change: per-warp sums
 
   // Sweep k gives this thread row g + k*NG; with NG*S = NT its piece is number tid + NT*k of
   // the row-major tile and its block's scale code is number tid/LPB + k*NT/LPB.
@@ -323,7 +326,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     constexpr bool INIT = decltype(init_tag)::value;
     constexpr bool EMIT = decltype(emit_tag)::value;
     float2 accN[8], accD[8], accS[INIT ? 8 : 1];
-    float2 accQd = make_float2(0.f, 0.f), accQp = make_float2(0.f, 0.f);   // QCH
+    float2 accQd = make_float2(0.f, 0.f), accQp = make_float2(0.f, 0.f);   // Q-change
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       accN[p] = make_float2(0.f, 0.f);
@@ -374,8 +377,8 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
         else q[p] = quant2_value<ELEM>(x);
       }
-      if constexpr (QCH && !INIT) {
-        if (t >= 2) {
+      if constexpr (EXT && !INIT) {
+        if (qch && t >= 2) {
           // q of the previous iteration, from its (r, c)
           const ScaleVal sp = scale_decode<SCALE>(pcode_at(k), tbl);
           const float2 irp = make_float2(sp.ir, sp.ir);
@@ -436,7 +439,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
       if (lib == 0) {
         set_code(k, sc.code);
-        if constexpr (QCH && !INIT) set_pcode(k, old_code);
+        if constexpr (EXT && !INIT) {
+          if (qch) set_pcode(k, old_code);
+        }
       }
 
       // c-step partial sums with the new r
@@ -465,7 +470,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     if (INIT && bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
 
     // ---- Q-change sums of this pass: per warp (exact), summed by thread 0 below
-    if constexpr (QCH) {
+    if (qch) {
       double qd = (double)accQd.x + (double)accQd.y, qp = (double)accQp.x + (double)accQp.y;
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) {
@@ -496,7 +501,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         const int j = warp * 16 + lane;
         const double Nj = nd;
         float cj = cvec[j];
-        if constexpr (QCH && !INIT) picvec[j] = icvec[j];   // 1/c of this pass's Q-step
+        if (!INIT && qch) picvec[j] = icvec[j];   // 1/c of this pass's Q-step
         if (!INIT && upd_c && Dj > 0.0) {
           cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
           cvec[j] = cj;
@@ -528,7 +533,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
       M.ws_err[(int64_t)t * tiles + tile] = e;
       if constexpr (INIT) M.ws_wsq[tile] = q2;
-      if constexpr (QCH) {
+      if (qch) {
         double qd = 0.0, qp = 0.0;
 #pragma unroll
         for (int i = 0; i < NWARP; ++i) {
@@ -550,9 +555,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   }
 }
 
-template <int ELEM, int SCALE, int LPB, int S, bool F32IN, bool QCH>
+template <int ELEM, int SCALE, int LPB, int S, bool F32IN, bool EXT>
 cudaError_t launch_one(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
-  auto kern = solve_kernel<ELEM, SCALE, LPB, S, F32IN, QCH>;
+  auto kern = solve_kernel<ELEM, SCALE, LPB, S, F32IN, EXT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)p.smem);
   if (e != cudaSuccess) return e;
@@ -565,42 +570,42 @@ cudaError_t launch_one(const SolveLaunch& L, int count, const SolvePlan& p, cuda
 }
 
 // tile width 16*S, S a power of two from LPB (one format block) to 8
-template <int ELEM, int SCALE, int LPB, bool F32IN, bool QCH>
+template <int ELEM, int SCALE, int LPB, bool F32IN, bool EXT>
 cudaError_t launch_s(const SolveLaunch& L, int count, const SolvePlan& p, cudaStream_t st) {
   switch (p.S) {
     case 1:
-      if constexpr (LPB <= 1) return launch_one<ELEM, SCALE, LPB, 1, F32IN, QCH>(L, count, p, st);
+      if constexpr (LPB <= 1) return launch_one<ELEM, SCALE, LPB, 1, F32IN, EXT>(L, count, p, st);
       break;
     case 2:
-      if constexpr (LPB <= 2) return launch_one<ELEM, SCALE, LPB, 2, F32IN, QCH>(L, count, p, st);
+      if constexpr (LPB <= 2) return launch_one<ELEM, SCALE, LPB, 2, F32IN, EXT>(L, count, p, st);
       break;
     case 4:
-      if constexpr (LPB <= 4) return launch_one<ELEM, SCALE, LPB, 4, F32IN, QCH>(L, count, p, st);
+      if constexpr (LPB <= 4) return launch_one<ELEM, SCALE, LPB, 4, F32IN, EXT>(L, count, p, st);
       break;
-    case 8: return launch_one<ELEM, SCALE, LPB, 8, F32IN, QCH>(L, count, p, st);
+    case 8: return launch_one<ELEM, SCALE, LPB, 8, F32IN, EXT>(L, count, p, st);
     default: break;
   }
   return cudaErrorInvalidValue;
 }
 
-template <int ELEM, int SCALE, int LPB, bool QCH>
+template <int ELEM, int SCALE, int LPB, bool EXT>
 cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const SolvePlan& p,
                          cudaStream_t st) {
-  return esize == 4 ? launch_s<ELEM, SCALE, LPB, true, QCH>(L, count, p, st)
-                    : launch_s<ELEM, SCALE, LPB, false, QCH>(L, count, p, st);
+  return esize == 4 ? launch_s<ELEM, SCALE, LPB, true, EXT>(L, count, p, st)
+                    : launch_s<ELEM, SCALE, LPB, false, EXT>(L, count, p, st);
 }
 
 // every format (kind as in dq.h; INT4 group 64 or 128)
-template <bool QCH>
+template <bool EXT>
 cudaError_t launch_solve_formats(const SolveLaunch& L, int count, int kind, int group,
                                  int esize, const SolvePlan& p, cudaStream_t s) {
   switch (kind) {
     case 0:
-      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4, QCH>(L, count, esize, p, s);
-      return launch_dtype<ELEM_INT4, SCALE_BF16, 8, QCH>(L, count, esize, p, s);
-    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, QCH>(L, count, esize, p, s);
-    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, QCH>(L, count, esize, p, s);
-    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, QCH>(L, count, esize, p, s);
+      if (group == 64) return launch_dtype<ELEM_INT4, SCALE_BF16, 4, EXT>(L, count, esize, p, s);
+      return launch_dtype<ELEM_INT4, SCALE_BF16, 8, EXT>(L, count, esize, p, s);
+    case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, EXT>(L, count, esize, p, s);
+    case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, EXT>(L, count, esize, p, s);
+    case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, EXT>(L, count, esize, p, s);
     default: return cudaErrorInvalidValue;
   }
 }
