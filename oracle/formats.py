@@ -1,7 +1,8 @@
-"""4-bit element grids and block-scale sets as explicit value tables (oracle; test only).
+"""Element grids and block-scale sets as explicit value tables (oracle; test only).
 
 The DualQuant pages name the formats (INT4 grouped, MXINT4, MXFP4, NVFP4 with E4M3 block
-scales and an FP32 tensor scale) but not their bit layouts; the tables below follow the
+scales and an FP32 tensor scale; the 8-bit appendix table: INT8 G=128 and MXINT8 G=32) but
+not their bit layouts; the tables below follow the
 public OCP Microscaling v1.0 definitions (E2M1 elements, E8M0 scales) and the usual FP8
 E4M3 ("FN": no infinities, 0x7F is NaN) definition. Every rounding is "nearest value in the
 table", with the tie rule stated beside it, computed in binary64 on a binary32 input, so the
@@ -35,7 +36,7 @@ BF16_MAX_BITS = 0x7F7F              # largest finite bf16
 E8M0_KMIN, E8M0_KMAX = -127, 127
 NVFP4_TENSOR_DIV = 6.0 * 448.0      # E2M1 max times E4M3 max
 
-FORMAT_KINDS = ("INT4", "MXINT4", "MXFP4", "NVFP4")
+FORMAT_KINDS = ("INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8")
 
 
 @dataclass(frozen=True)
@@ -45,20 +46,28 @@ class Format:
 
     @property
     def elem(self) -> str:
-        return "int4" if self.kind in ("INT4", "MXINT4") else "e2m1"
+        return {"INT4": "int4", "MXINT4": "int4", "MXFP4": "e2m1", "NVFP4": "e2m1",
+                "INT8": "int8", "MXINT8": "int8"}[self.kind]
 
     @property
     def scale(self) -> str:
-        return {"INT4": "bf16", "MXINT4": "e8m0", "MXFP4": "e8m0", "NVFP4": "e4m3"}[self.kind]
+        return {"INT4": "bf16", "MXINT4": "e8m0", "MXFP4": "e8m0", "NVFP4": "e4m3",
+                "INT8": "bf16", "MXINT8": "e8m0"}[self.kind]
 
     @property
     def qmax(self) -> float:
-        return 7.0 if self.elem == "int4" else 6.0
+        return {"int4": 7.0, "e2m1": 6.0, "int8": 127.0}[self.elem]
+
+    @property
+    def bits(self) -> int:
+        """Bits per element code: 4 (two codes per byte) or 8 (one byte, two's complement)."""
+        return 8 if self.elem == "int8" else 4
 
 
 def make_format(kind: str, block: int | None = None) -> Format:
-    """The four 4-bit formats; `block` overrides the block length (tests use tiny blocks)."""
-    default = {"INT4": 128, "MXINT4": 32, "MXFP4": 32, "NVFP4": 16}[kind]
+    """The formats by name; `block` overrides the block length (tests use tiny blocks)."""
+    default = {"INT4": 128, "MXINT4": 32, "MXFP4": 32, "NVFP4": 16, "INT8": 128,
+               "MXINT8": 32}[kind]
     return Format(kind, int(block if block is not None else default))
 
 
@@ -85,11 +94,15 @@ def round_elem(x32: np.ndarray, fmt: Format):
     """RNE of binary32 x onto the element grid, saturating.
 
     Returns (codes uint8, values float64). INT4 codes are two's-complement nibbles of the
-    integer; E2M1 codes are sign<<3 | magnitude code, the sign taken from x's sign bit."""
+    integer, INT8 codes its two's-complement byte (symmetric grid -127..127, like INT4's
+    -7..7: the most negative code is never produced); E2M1 codes are sign<<3 | magnitude
+    code, the sign taken from x's sign bit."""
     x = np.asarray(x32, dtype=np.float32).astype(np.float64)
-    if fmt.elem == "int4":
-        q = np.clip(np.rint(x), -7.0, 7.0)           # np.rint rounds half to even
-        codes = (q.astype(np.int64) & 0xF).astype(np.uint8)
+    if fmt.elem in ("int4", "int8"):
+        qm = fmt.qmax
+        q = np.clip(np.rint(x), -qm, qm)             # np.rint rounds half to even
+        mask = 0xF if fmt.elem == "int4" else 0xFF
+        codes = (q.astype(np.int64) & mask).astype(np.uint8)
         return codes, q
     neg = np.signbit(x)
     idx = _nearest_sorted(E2M1_MAG, np.abs(x))
@@ -102,6 +115,8 @@ def decode_elem(codes: np.ndarray, fmt: Format) -> np.ndarray:
     codes = np.asarray(codes, dtype=np.int64)
     if fmt.elem == "int4":
         return np.where(codes >= 8, codes - 16, codes).astype(np.float64)
+    if fmt.elem == "int8":
+        return np.where(codes >= 128, codes - 256, codes).astype(np.float64)
     mag = E2M1_MAG[codes & 7]
     return np.where(codes & 8, -mag, mag)
 
@@ -180,14 +195,19 @@ def decode_scale(codes: np.ndarray, fmt: Format, s_t: np.float32 | None = None):
         np.float32)
 
 
-def pack_codes(codes: np.ndarray) -> np.ndarray:
-    """[rows, n] 4-bit codes -> [rows, n/2] bytes, low nibble = even column."""
+def pack_codes(codes: np.ndarray, bits: int = 4) -> np.ndarray:
+    """[rows, n] 4-bit codes -> [rows, n/2] bytes, low nibble = even column (8-bit codes
+    are stored one per byte, unchanged)."""
     codes = np.asarray(codes, dtype=np.uint8)
+    if bits == 8:
+        return codes.copy()
     return (codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)
 
 
-def unpack_codes(packed: np.ndarray) -> np.ndarray:
+def unpack_codes(packed: np.ndarray, bits: int = 4) -> np.ndarray:
     packed = np.asarray(packed, dtype=np.uint8)
+    if bits == 8:
+        return packed.copy()
     out = np.empty((packed.shape[0], packed.shape[1] * 2), dtype=np.uint8)
     out[:, 0::2] = packed & 0xF
     out[:, 1::2] = packed >> 4

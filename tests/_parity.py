@@ -29,7 +29,8 @@ def oracle_format(name_or_spec):
     if isinstance(name_or_spec, str):
         kind, group = {"INT4": ("INT4", 128), "INT4_G64": ("INT4", 64),
                        "MXINT4": ("MXINT4", 32), "MXFP4": ("MXFP4", 32),
-                       "NVFP4": ("NVFP4", 16)}[name_or_spec]
+                       "NVFP4": ("NVFP4", 16), "INT8": ("INT8", 128),
+                       "INT8_G64": ("INT8", 64), "MXINT8": ("MXINT8", 32)}[name_or_spec]
     else:
         kind, group = name_or_spec.kind, name_or_spec.group
     return F.make_format(kind, group)
@@ -46,7 +47,7 @@ def to_host(out: dict) -> dict:
 
 def grid_index(q: np.ndarray, fmt) -> np.ndarray:
     """Position of each element value on the signed grid (-0 and +0 coincide)."""
-    if fmt.elem == "int4":
+    if fmt.elem in ("int4", "int8"):
         return np.rint(q).astype(np.int64)
     mag = np.abs(q)
     idx = np.searchsorted(F.E2M1_MAG, mag)
@@ -67,7 +68,7 @@ def scale_step(code_a: np.ndarray, code_b: np.ndarray, fmt) -> np.ndarray:
 
 def compare_solve(h: dict, ora: dict, fmt, *, exact: bool = False, label: str = "") -> dict:
     """Assert the parity bar; return the measured agreement figures."""
-    codes_g = F.unpack_codes(h["q_packed"])
+    codes_g = F.unpack_codes(h["q_packed"], fmt.bits)
     codes_o = ora["codes"]
     qg = F.decode_elem(codes_g, fmt)
     qo = ora["q"]

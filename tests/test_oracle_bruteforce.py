@@ -13,13 +13,13 @@ import pytest
 from oracle import formats as F
 from oracle import solver as S
 
-KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4"]
+KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8"]
 M, N, B = 4, 8, 4
 
 
 def _grid(fmt):
-    if fmt.elem == "int4":
-        return np.arange(-7, 8, dtype=np.float64)
+    if fmt.elem in ("int4", "int8"):
+        return np.arange(-fmt.qmax, fmt.qmax + 1, dtype=np.float64)
     return np.concatenate([-F.E2M1_MAG[:0:-1], F.E2M1_MAG])
 
 

@@ -173,6 +173,31 @@ def test_int4_codes_are_twos_complement():
     np.testing.assert_array_equal(F.decode_elem(codes, fmt), q)
 
 
+def test_int8_round_matches_torch_and_brute_force():
+    """INT8 elements (the 8-bit appendix table): RNE onto -127..127, saturating; torch's
+    round (half to even) and clamp, and the nearest-integer brute force, agree."""
+    for kind in ("INT8", "MXINT8"):
+        fmt = F.make_format(kind)
+        rng = np.random.default_rng(6)
+        x = np.concatenate([rng.uniform(-140, 140, 4000), np.arange(-130, 130) + 0.5,
+                            [127.5, -127.5, 128.0, -128.0, 1e30, -1e30]]).astype(np.float32)
+        codes, got = F.round_elem(x, fmt)
+        ref_t = torch.clamp(torch.round(torch.from_numpy(x).double()), -127, 127).numpy()
+        np.testing.assert_array_equal(got, ref_t)
+        np.testing.assert_array_equal(got[:3000], _brute_round(x[:3000], range(-127, 128), float))
+        # codes are the two's-complement bytes of the integers (torch's int8 view)
+        tb = torch.from_numpy(got.astype(np.int8)).view(torch.uint8).numpy()
+        np.testing.assert_array_equal(codes, tb)
+        np.testing.assert_array_equal(F.decode_elem(codes, fmt), got)
+        assert 0x80 not in set(codes.tolist())          # -128 is never produced
+
+
+def test_int8_codes_are_stored_one_per_byte():
+    codes = np.arange(256, dtype=np.uint8).reshape(4, 64)
+    np.testing.assert_array_equal(F.pack_codes(codes, 8), codes)
+    np.testing.assert_array_equal(F.unpack_codes(F.pack_codes(codes, 8), 8), codes)
+
+
 def test_pack_roundtrip_low_nibble_even_column():
     rng = np.random.default_rng(5)
     codes = rng.integers(0, 16, (3, 8)).astype(np.uint8)

@@ -16,7 +16,7 @@ from oracle import formats as F
 from oracle import solver as S
 from oracle.actquant import act_quant, rescale
 
-KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4"]
+KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8"]
 
 
 def _small(kind, seed=0, m=96, n=256):
@@ -53,17 +53,17 @@ def _rtn_reference(W, kind):
     m, n = W.shape
     a = Wt.reshape(m, n // fmt.block, fmt.block).abs().amax(dim=2)
     v = a / fmt.qmax
-    if kind == "INT4":
+    if kind in ("INT4", "INT8"):
         s = v.to(torch.bfloat16).to(torch.float64)
-    elif kind in ("MXINT4", "MXFP4"):
+    elif kind in ("MXINT4", "MXFP4", "MXINT8"):
         s = v.to(torch.float8_e8m0fnu).to(torch.float64)
     else:
         st = torch.tensor(float(a.max()), dtype=torch.float32) / 2688.0
         e = (v / st).to(torch.float8_e4m3fn).to(torch.float32)
         s = (st * e).to(torch.float64)
     x = Wt.to(torch.float64) / s.repeat_interleave(fmt.block, dim=1)
-    if fmt.elem == "int4":
-        q = torch.clamp(torch.round(x), -7, 7)
+    if fmt.elem in ("int4", "int8"):
+        q = torch.clamp(torch.round(x), -fmt.qmax, fmt.qmax)
     else:
         grid = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=torch.float64)
         d = (x.abs().unsqueeze(-1) - grid).abs()
@@ -80,7 +80,7 @@ def test_iteration0_is_single_scale_rtn(kind):
     np.testing.assert_array_equal(out["r"].astype(np.float64), s_ref)
     np.testing.assert_array_equal(out["c"], np.ones(W.shape[1], np.float32))
     diff = out["q"] != q_ref
-    if fmt.elem == "int4":
+    if fmt.elem in ("int4", "int8"):
         mids = np.abs(np.abs(x_ref) - (np.floor(np.abs(x_ref)) + 0.5))
     else:
         g = F.E2M1_MAG
@@ -102,7 +102,8 @@ def test_exact_model_is_a_fixed_point(kind):
         r = (2.0 ** rng.integers(-9, -4, (m, n // fmt.block))).astype(np.float32)
     else:
         r = (s_t * F.E4M3_POS[rng.integers(40, 90, (m, n // fmt.block))]).astype(np.float32)
-    grid = np.arange(-7, 8) if fmt.elem == "int4" else np.concatenate(
+    qm = int(fmt.qmax)
+    grid = np.arange(-qm, qm + 1) if fmt.elem != "e2m1" else np.concatenate(
         [-F.E2M1_MAG[:0:-1], F.E2M1_MAG])
     q = rng.choice(grid[grid != 0], (m, n)).astype(np.float64)
     c = (rng.integers(4, 16, n) / 8.0).astype(np.float32)     # few mantissa bits

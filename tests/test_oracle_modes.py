@@ -14,7 +14,7 @@ import pytest
 from oracle import formats as F
 from oracle import solver as S
 
-KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4"]
+KINDS = ["INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8"]
 
 
 def _small(seed, m=24, n=64):
@@ -57,7 +57,8 @@ def test_single_side_modes_keep_the_other_scale_and_stay_monotone(kind, update):
 def test_row_only_update_is_the_best_admissible_scale(kind):
     """One row-only iteration from RTN: each block's new scale minimises
     sum_b (W - r q c)^2 over all admissible values (q and c = 1 fixed)."""
-    fmt = F.make_format(kind, {"INT4": 32, "MXINT4": 32, "MXFP4": 32, "NVFP4": 16}[kind])
+    fmt = F.make_format(kind, {"INT4": 32, "MXINT4": 32, "MXFP4": 32, "NVFP4": 16, "INT8": 32,
+                               "MXINT8": 32}[kind])
     W = _small(11, 6, 64)
     out = S.solve(W, fmt, 1, update="row")
     q, r = out["q"], out["r"].astype(np.float64)
