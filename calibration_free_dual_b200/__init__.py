@@ -10,8 +10,9 @@ The C ABI is reachable under its own names (`dq_solve`, `dq_solve_batched`,
 workspace with torch and call them.
 """
 from . import _lib
-from ._lib import (DQ_OK, DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4, DQ_F32, DQ_BF16,  # noqa: F401
-                   DQ_CODEC_INT4, DQ_CODEC_E2M1, DQ_CODEC_E4M3, DQ_CODEC_E8M0, DQ_CODEC_BF16,
+from ._lib import (DQ_OK, DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4, DQ_INT8,  # noqa: F401
+                   DQ_MXINT8, DQ_F32, DQ_BF16, DQ_CODEC_INT4, DQ_CODEC_E2M1, DQ_CODEC_E4M3,
+                   DQ_CODEC_E8M0, DQ_CODEC_BF16, DQ_CODEC_INT8,
                    DQ_UPDATE_BOTH, DQ_UPDATE_ROW_ONLY, DQ_UPDATE_COL_ONLY,
                    dq_format, dq_matrix, dq_solve_options)
 from .api import (DQError, FORMATS, fmt_of, solve, solve_batched, act_quant, encode,  # noqa: F401

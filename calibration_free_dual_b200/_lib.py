@@ -10,9 +10,10 @@ c_void_p, c_int32, c_int64, c_size_t = ctypes.c_void_p, ctypes.c_int32, ctypes.c
 
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_SHAPE, DQ_ERR_DTYPE, DQ_ERR_WORKSPACE = 0, 1, 2, 3, 4
 DQ_ERR_NONFINITE, DQ_ERR_TIMEOUT, DQ_ERR_CUDA, DQ_ERR_UNSUPPORTED = 5, 6, 7, 8
-DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4 = 0, 1, 2, 3
+DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4, DQ_INT8, DQ_MXINT8 = 0, 1, 2, 3, 4, 5
 DQ_F32, DQ_BF16 = 0, 1
 DQ_CODEC_INT4, DQ_CODEC_E2M1, DQ_CODEC_E4M3, DQ_CODEC_E8M0, DQ_CODEC_BF16 = 0, 1, 2, 3, 4
+DQ_CODEC_INT8 = 5
 DQ_NOALLOC_SCRATCH_BYTES = 4 << 20
 DQ_UPDATE_BOTH, DQ_UPDATE_ROW_ONLY, DQ_UPDATE_COL_ONLY = 0, 1, 2
 

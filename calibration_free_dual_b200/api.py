@@ -17,9 +17,17 @@ FORMATS = {
     "INT4": (_lib.DQ_INT4, 128), "INT4_G128": (_lib.DQ_INT4, 128),
     "INT4_G64": (_lib.DQ_INT4, 64), "MXINT4": (_lib.DQ_MXINT4, 32),
     "MXFP4": (_lib.DQ_MXFP4, 32), "NVFP4": (_lib.DQ_NVFP4, 16),
+    "INT8": (_lib.DQ_INT8, 128), "INT8_G128": (_lib.DQ_INT8, 128),
+    "INT8_G64": (_lib.DQ_INT8, 64), "MXINT8": (_lib.DQ_MXINT8, 32),
 }
 _KIND_NAMES = {"INT4": _lib.DQ_INT4, "MXINT4": _lib.DQ_MXINT4, "MXFP4": _lib.DQ_MXFP4,
-               "NVFP4": _lib.DQ_NVFP4}
+               "NVFP4": _lib.DQ_NVFP4, "INT8": _lib.DQ_INT8, "MXINT8": _lib.DQ_MXINT8}
+_BF16_SCALES = (_lib.DQ_INT4, _lib.DQ_INT8)
+
+
+def _code_cols(f, n: int) -> int:
+    """Bytes of element codes per row: two 4-bit codes per byte, one 8-bit code."""
+    return n if f.kind in (_lib.DQ_INT8, _lib.DQ_MXINT8) else n // 2
 
 
 class DQError(RuntimeError):
@@ -75,9 +83,9 @@ def _need_cuda(t: torch.Tensor, name: str) -> None:
 def solve_outputs(m: int, n: int, fmt, iters: int, device) -> dict:
     f = fmt_of(fmt)
     B = f.group
-    sdt = torch.int16 if f.kind == _lib.DQ_INT4 else torch.uint8
+    sdt = torch.int16 if f.kind in _BF16_SCALES else torch.uint8
     return dict(
-        q_packed=torch.empty((m, n // 2), dtype=torch.uint8, device=device),
+        q_packed=torch.empty((m, _code_cols(f, n)), dtype=torch.uint8, device=device),
         r=torch.empty((m, n // B), dtype=torch.float32, device=device),
         c=torch.empty((n,), dtype=torch.float32, device=device),
         block_scales=torch.empty((m, n // B), dtype=sdt, device=device),
@@ -185,8 +193,8 @@ def act_quant(X: torch.Tensor, fmt, c: torch.Tensor | None = None, stream=None) 
     f = fmt_of(fmt)
     T, n = X.shape
     B = f.group
-    sdt = torch.int16 if f.kind == _lib.DQ_INT4 else torch.uint8
-    o = dict(x_packed=torch.empty((T, n // 2), dtype=torch.uint8, device=X.device),
+    sdt = torch.int16 if f.kind in _BF16_SCALES else torch.uint8
+    o = dict(x_packed=torch.empty((T, _code_cols(f, n)), dtype=torch.uint8, device=X.device),
              scales=torch.empty((T, n // B), dtype=sdt, device=X.device),
              tensor_scale=torch.empty((1,), dtype=torch.float32, device=X.device))
     lib = _lib.get()

@@ -1,4 +1,5 @@
-// dq_act.cu — activation rescale by the solver's column scales + 4-bit block quantization.
+// dq_act.cu — activation rescale by the solver's column scales + block quantization (4-bit
+// formats; INT8 and MXINT8 for the appendix's 8-bit W8A8 setting).
 //
 // DualQuant ("DualQuant: Dual-scale Calibration-free Weight-and-Activation Quantization for
 // LLMs", Abstract; appendix Table 11, activation quantization including beta; appendix
@@ -82,8 +83,9 @@ __global__ void act_amax_kernel(const ActLaunch A) {
 template <int ELEM, int SCALE, int B, bool F32IN>
 __global__ void act_quant_kernel(const ActLaunch A) {
   constexpr int LB = B / 8;                       // lanes per block
-  constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
+  constexpr float QMAX = elem_qmax<ELEM>();
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
+  constexpr bool BYTE_CODES = (ELEM == ELEM_INT8);         // one code byte per element
   const int lane = threadIdx.x & 31;
   const int64_t warp0 = (int64_t)blockIdx.x * ACT_WARPS + threadIdx.x / 32;
   const int64_t nwarps = (int64_t)gridDim.x * ACT_WARPS;
@@ -92,7 +94,7 @@ __global__ void act_quant_kernel(const ActLaunch A) {
     s_t = nvfp4_tensor_scale(__uint_as_float(*A.amax_bits));
     if (blockIdx.x == 0 && threadIdx.x == 0 && A.tensor_scale != nullptr) *A.tensor_scale = s_t;
   }
-  const int64_t nb = A.n / B, nh = A.n / 2;
+  const int64_t nb = A.n / B, qpitch = BYTE_CODES ? A.n : A.n / 2;
   bool bad = false;
   for (int64_t row = warp0; row < A.tokens; row += nwarps) {
     for (int64_t base = 0; base < A.n; base += 256) {
@@ -121,16 +123,20 @@ __global__ void act_quant_kernel(const ActLaunch A) {
         code = sv.code;
         inv = sv.ir;
       }
-      uint32_t packed = 0;
+      uint64_t packed = 0;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         float2 q;
         uint32_t cb = quant2<ELEM>(make_float2(__fmul_rn(x[2 * k], inv), __fmul_rn(x[2 * k + 1], inv)), q);
-        packed |= (cb & 0xFFu) << (8 * k);
+        if constexpr (BYTE_CODES) packed |= (uint64_t)(cb & 0xFFFFu) << (16 * k);
+        else packed |= (uint64_t)(cb & 0xFFu) << (8 * k);
       }
       if (valid) {
         if (a == 0.0f) packed = 0;   // all-zero block: code 0 (also for -0 inputs)
-        *reinterpret_cast<uint32_t*>(A.x_packed + row * nh + col / 2) = packed;
+        if constexpr (BYTE_CODES)
+          *reinterpret_cast<uint64_t*>(A.x_packed + row * qpitch + col) = packed;
+        else
+          *reinterpret_cast<uint32_t*>(A.x_packed + row * qpitch + col / 2) = (uint32_t)packed;
         if ((lane % LB) == 0) {
           if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(A.scales)[row * nb + col / B] = (uint16_t)code;
           else reinterpret_cast<uint8_t*>(A.scales)[row * nb + col / B] = (uint8_t)code;
@@ -169,6 +175,10 @@ cudaError_t launch_act(const ActLaunch& A, int kind, int group, int esize, cudaS
     case 1: return launch_fmt<ELEM_INT4, SCALE_E8M0, 32>(A, esize, s);
     case 2: return launch_fmt<ELEM_E2M1, SCALE_E8M0, 32>(A, esize, s);
     case 3: return launch_fmt<ELEM_E2M1, SCALE_E4M3, 16>(A, esize, s);
+    case 4:
+      if (group == 64) return launch_fmt<ELEM_INT8, SCALE_BF16, 64>(A, esize, s);
+      return launch_fmt<ELEM_INT8, SCALE_BF16, 128>(A, esize, s);
+    case 5: return launch_fmt<ELEM_INT8, SCALE_E8M0, 32>(A, esize, s);
     default: return cudaErrorInvalidValue;
   }
 }

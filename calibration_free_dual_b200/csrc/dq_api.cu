@@ -50,7 +50,7 @@ size_t per_matrix_ws(int tiles, int iters, bool qch) {
 size_t amax_head(int64_t count) { return dq::align_up(sizeof(unsigned) * (size_t)count, 256); }
 
 dq_status check_format(dq_format f) {
-  if (f.kind < DQ_INT4 || f.kind > DQ_NVFP4) return DQ_ERR_DTYPE;
+  if (f.kind < DQ_INT4 || f.kind > DQ_MXINT8) return DQ_ERR_DTYPE;
   if (dq::fmt_block(f.kind, f.group) == 0) return DQ_ERR_DTYPE;
   return DQ_OK;
 }
@@ -160,7 +160,9 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
       return DQ_ERR_INVALID_ARG;
     if (fmt.kind == DQ_NVFP4 && d.tensor_scale == nullptr) return DQ_ERR_INVALID_ARG;
     if (!aligned16(d.W) || (d.ldw * esize) % 16 != 0) return DQ_ERR_INVALID_ARG;
-    if ((reinterpret_cast<uintptr_t>(d.q_packed) & 7u) != 0) return DQ_ERR_INVALID_ARG;
+    // 4-bit codes are stored 8 bytes per thread, 8-bit codes 16
+    const uintptr_t qalign = dq::fmt_elem_bits(fmt.kind) == 8 ? 15u : 7u;
+    if ((reinterpret_cast<uintptr_t>(d.q_packed) & qalign) != 0) return DQ_ERR_INVALID_ARG;
     ms[i] = d.m;
     ns[i] = d.n;
   }
@@ -252,10 +254,12 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
       if (fmt.kind == DQ_NVFP4) {
         if ((st = from_cuda(dq::launch_solve_amax(L, c, esize, s))) != DQ_OK) return st;
       }
+      const bool ext = qch || update != DQ_UPDATE_BOTH;
       const cudaError_t e =
-          (qch || update != DQ_UPDATE_BOTH)
-              ? dq::launch_solve_ext(L, c, fmt.kind, fmt.group, esize, plan, s)
-              : dq::launch_solve(L, c, fmt.kind, fmt.group, esize, plan, s);
+          dq::fmt_elem_bits(fmt.kind) == 8
+              ? dq::launch_solve_8bit(L, c, fmt.kind, fmt.group, esize, plan, ext, s)
+              : (ext ? dq::launch_solve_ext(L, c, fmt.kind, fmt.group, esize, plan, s)
+                     : dq::launch_solve(L, c, fmt.kind, fmt.group, esize, plan, s));
       if ((st = from_cuda(e)) != DQ_OK) return st;
     }
   }
@@ -322,7 +326,8 @@ dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, 
   if (fmt.kind == DQ_NVFP4 && tensor_scale == nullptr) return DQ_ERR_INVALID_ARG;
   if (!aligned16(X) || (ldx * esize) % 16 != 0) return DQ_ERR_INVALID_ARG;
   if (c != nullptr && !aligned16(c)) return DQ_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x_packed) & 3u) != 0) return DQ_ERR_INVALID_ARG;
+  const uintptr_t xalign = dq::fmt_elem_bits(fmt.kind) == 8 ? 7u : 3u;
+  if ((reinterpret_cast<uintptr_t>(x_packed) & xalign) != 0) return DQ_ERR_INVALID_ARG;
   if (workspace == nullptr || workspace_bytes < dq_act_quant_workspace_bytes(tokens, n, fmt))
     return DQ_ERR_WORKSPACE;
   unsigned* errp = nullptr;
@@ -346,14 +351,14 @@ dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, 
 }
 
 dq_status dq_encode(const float* x, int64_t count, int32_t codec, void* codes, void* stream) {
-  if (codec < DQ_CODEC_INT4 || codec > DQ_CODEC_BF16) return DQ_ERR_DTYPE;
+  if (codec < DQ_CODEC_INT4 || codec > DQ_CODEC_INT8) return DQ_ERR_DTYPE;
   if (count < 0) return DQ_ERR_INVALID_ARG;
   if (count > 0 && (x == nullptr || codes == nullptr)) return DQ_ERR_INVALID_ARG;
   return from_cuda(dq::launch_encode(x, count, codec, codes, static_cast<cudaStream_t>(stream)));
 }
 
 dq_status dq_decode(const void* codes, int64_t count, int32_t codec, float* x, void* stream) {
-  if (codec < DQ_CODEC_INT4 || codec > DQ_CODEC_BF16) return DQ_ERR_DTYPE;
+  if (codec < DQ_CODEC_INT4 || codec > DQ_CODEC_INT8) return DQ_ERR_DTYPE;
   if (count < 0) return DQ_ERR_INVALID_ARG;
   if (count > 0 && (x == nullptr || codes == nullptr)) return DQ_ERR_INVALID_ARG;
   return from_cuda(dq::launch_decode(codes, count, codec, x, static_cast<cudaStream_t>(stream)));

@@ -23,6 +23,7 @@ __global__ void encode_kernel(const float* x, int64_t count, int codec, void* co
       }
       case 3: reinterpret_cast<uint8_t*>(codes)[i] = (uint8_t)e8m0_encode(v); break;
       case 4: reinterpret_cast<uint16_t*>(codes)[i] = (uint16_t)bf16_rn_bits(v); break;
+      case 5: reinterpret_cast<uint8_t*>(codes)[i] = (uint8_t)int8_code(int8_round(v)); break;
       default: break;
     }
   }
@@ -47,6 +48,7 @@ __global__ void decode_kernel(const void* codes, int64_t count, int codec, float
       }
       case 3: v = e8m0_decode(reinterpret_cast<const uint8_t*>(codes)[i]); break;
       case 4: v = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(codes)[i] << 16); break;
+      case 5: v = (float)reinterpret_cast<const int8_t*>(codes)[i]; break;
       default: break;
     }
     x[i] = v;

@@ -1,6 +1,7 @@
 // dq_device.cuh — device-side codecs and projections shared by the DualQuant kernels.
 //
-// Element grids: INT4 (-7..7) and E2M1 (OCP MX v1.0 FP4); block scales: bf16, E8M0 and
+// Element grids: INT4 (-7..7), INT8 (-127..127) and E2M1 (OCP MX v1.0 FP4); block scales:
+// bf16, E8M0 and
 // E4M3 (FN) times an fp32 tensor scale. Every rounding is round-to-nearest-even on a binary32
 // input (E8M0: nearest power of two, tie up), saturating at the grid's largest magnitude.
 // Pi_S maps a scale to the nearest member of the format's set of representable block
@@ -15,7 +16,13 @@
 
 namespace dq {
 
-enum Elem : int { ELEM_INT4 = 0, ELEM_E2M1 = 1 };
+enum Elem : int { ELEM_INT4 = 0, ELEM_E2M1 = 1, ELEM_INT8 = 2 };
+
+// largest element magnitude of a grid
+template <int ELEM>
+__host__ __device__ constexpr float elem_qmax() {
+  return ELEM == ELEM_INT4 ? 7.0f : (ELEM == ELEM_INT8 ? 127.0f : 6.0f);
+}
 enum Scale : int { SCALE_BF16 = 0, SCALE_E8M0 = 1, SCALE_E4M3 = 2 };
 
 // error bits of the per-device error word
@@ -51,19 +58,28 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
   return __half22float2(hv);
 }
 
-// ------------------------------------------------------------------ INT4 elements
+// ------------------------------------------------------------------ INT4 / INT8 elements
 __device__ __forceinline__ float int4_round(float x) {
   return fminf(fmaxf(rintf(x), -7.0f), 7.0f);
 }
 __device__ __forceinline__ uint32_t int4_code(float q) { return ((int)q) & 0xF; }
+__device__ __forceinline__ float int8_round(float x) {
+  return fminf(fmaxf(rintf(x), -127.0f), 127.0f);
+}
+__device__ __forceinline__ uint32_t int8_code(float q) { return ((int)q) & 0xFF; }
 
-// Quantize a pair on the element grid: values into q, code byte (low nibble = x.x).
+// Quantize a pair on the element grid: values into q; codes of x.x and x.y, x.x lowest:
+// one byte of two nibbles (4-bit grids) or two bytes (INT8).
 template <int ELEM>
 __device__ __forceinline__ uint32_t quant2(float2 x, float2& q) {
   if constexpr (ELEM == ELEM_E2M1) {
     uint32_t code = e2m1x2_encode(x.x, x.y);
     q = e2m1x2_decode(code);
     return code;
+  } else if constexpr (ELEM == ELEM_INT8) {
+    q.x = int8_round(x.x);
+    q.y = int8_round(x.y);
+    return int8_code(q.x) | (int8_code(q.y) << 8);
   } else {
     q.x = int4_round(x.x);
     q.y = int4_round(x.y);
@@ -82,6 +98,8 @@ __device__ __forceinline__ float2 quant2_value(float2 x) {
         : "=r"(h2) : "f"(x.x), "f"(x.y));
     __half2 hv = *reinterpret_cast<__half2*>(&h2);
     return __half22float2(hv);
+  } else if constexpr (ELEM == ELEM_INT8) {
+    return make_float2(int8_round(x.x), int8_round(x.y));
   } else {
     return make_float2(int4_round(x.x), int4_round(x.y));
   }

@@ -76,15 +76,17 @@ __host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, in
   return l;
 }
 
-// format helpers (kind as in dq.h)
+// format helpers (kind as in dq.h: INT4, MXINT4, MXFP4, NVFP4, INT8, MXINT8)
 inline int fmt_block(int kind, int group) {
   switch (kind) {
-    case 0: return (group == 64 || group == 128) ? group : 0;
-    case 1: case 2: return group == 32 ? 32 : 0;
+    case 0: case 4: return (group == 64 || group == 128) ? group : 0;
+    case 1: case 2: case 5: return group == 32 ? 32 : 0;
     case 3: return group == 16 ? 16 : 0;
     default: return 0;
   }
 }
+inline int fmt_scale_bytes(int kind) { return (kind == 0 || kind == 4) ? 2 : 1; }   // bf16: 2
+inline int fmt_elem_bits(int kind) { return kind >= 4 ? 8 : 4; }
 
 // measurement hooks (dq_api.cu)
 void count_launches(int n);
@@ -99,6 +101,11 @@ cudaError_t launch_solve(const SolveLaunch& L, int count, int kind, int group, i
 // the extended instantiation: update modes and the Q-change trace (L.upd_r, L.upd_c, L.qch)
 cudaError_t launch_solve_ext(const SolveLaunch& L, int count, int kind, int group, int esize,
                              const SolvePlan& p, cudaStream_t s);
+// the 8-bit formats (INT8, MXINT8), plain or extended
+cudaError_t launch_solve_8bit(const SolveLaunch& L, int count, int kind, int group, int esize,
+                              const SolvePlan& p, bool ext, cudaStream_t s);
+cudaError_t launch_solve_8bit_ext(const SolveLaunch& L, int count, int kind, int group,
+                                  int esize, const SolvePlan& p, cudaStream_t s);
 cudaError_t launch_solve_amax(const SolveLaunch& L, int count, int esize, cudaStream_t s);
 // qchange / ws_qch may be null (no Q-change trace)
 cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* const* ws_wsq,

@@ -108,7 +108,7 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, 
   const int B = fmt_block(kind, group);
   if (B == 0 || m <= 0 || n <= 0 || n % B || m > (1 << 24)) return false;
   const int LPB = B / 16;
-  const int scb = kind == 0 ? 2 : 1;
+  const int scb = fmt_scale_bytes(kind);
   int S = LPB;
   while (S < 8 && m * S < (int64_t)16 * SOLVE_NT && n % (32 * S) == 0) S *= 2;
   const int NG = SOLVE_NT / S;

@@ -142,7 +142,8 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   constexpr int NG = NT / S;             // rows covered by one sweep of all threads
   constexpr int ESZ = F32IN ? 4 : 2;
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
-  constexpr float QMAX = (ELEM == ELEM_INT4) ? 7.0f : 6.0f;
+  constexpr float QMAX = elem_qmax<ELEM>();
+  constexpr bool BYTE_CODES = (ELEM == ELEM_INT8);        // one code byte per element
   static_assert(NBLK * LPB == S && S >= 1 && S <= 8, "tile shape");
 
   const int m = L.m, n = L.n, T = L.T, tiles = L.tiles;
@@ -262,7 +263,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
   const int RPT = (m + NG - 1) / NG;       // sweeps per pass (uniform: shuffles below)
   const int KS = min(L.R / NG, RPT);       // sweeps served from shared memory
-  const int nh = n >> 1;
+  const int64_t qpitch = BYTE_CODES ? n : (n >> 1);         // code bytes per row
 
   // row piece of sweep k: shared memory (chunk h of piece tid + NT*k sits at
   // ESZ*(tid + NT*k) + (h ^ sw)), else L2, or zeros past the last row
@@ -369,12 +370,13 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
       float2 q[8];
-      uint32_t codes[2] = {0u, 0u};
+      uint32_t codes[4] = {0u, 0u, 0u, 0u};
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
         const float2 x = mul2(mul2(w[p], ic[p]), irr);
-        if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
+        if constexpr (EMIT && BYTE_CODES) codes[p >> 1] |= quant2<ELEM>(x, q[p]) << (16 * (p & 1));
+        else if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
         else q[p] = quant2_value<ELEM>(x);
       }
       if constexpr (EXT && !INIT) {
@@ -456,8 +458,13 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
       if constexpr (EMIT) {
         if (row < m) {
-          uint8_t* qp = M.q_packed + (int64_t)row * nh + (col0 + s * 16) / 2;
-          *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
+          if constexpr (BYTE_CODES) {
+            uint8_t* qp = M.q_packed + (int64_t)row * qpitch + col0 + s * 16;
+            *reinterpret_cast<uint4*>(qp) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+          } else {
+            uint8_t* qp = M.q_packed + (int64_t)row * qpitch + (col0 + s * 16) / 2;
+            *reinterpret_cast<uint2*>(qp) = make_uint2(codes[0], codes[1]);
+          }
           if (lib == 0) {
             const int64_t bi = (int64_t)row * nb + col0 / B + bl;
             M.r[bi] = sc.r;
@@ -595,7 +602,7 @@ cudaError_t launch_dtype(const SolveLaunch& L, int count, int esize, const Solve
                     : launch_s<ELEM, SCALE, LPB, false, EXT>(L, count, p, st);
 }
 
-// every format (kind as in dq.h; INT4 group 64 or 128)
+// the 4-bit formats (kind as in dq.h; INT4 group 64 or 128)
 template <bool EXT>
 cudaError_t launch_solve_formats(const SolveLaunch& L, int count, int kind, int group,
                                  int esize, const SolvePlan& p, cudaStream_t s) {
@@ -606,6 +613,19 @@ cudaError_t launch_solve_formats(const SolveLaunch& L, int count, int kind, int 
     case 1: return launch_dtype<ELEM_INT4, SCALE_E8M0, 2, EXT>(L, count, esize, p, s);
     case 2: return launch_dtype<ELEM_E2M1, SCALE_E8M0, 2, EXT>(L, count, esize, p, s);
     case 3: return launch_dtype<ELEM_E2M1, SCALE_E4M3, 1, EXT>(L, count, esize, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// the 8-bit formats: INT8 (group 64 or 128, bf16 scales), MXINT8 (32, E8M0)
+template <bool EXT>
+cudaError_t launch_solve_formats8(const SolveLaunch& L, int count, int kind, int group,
+                                  int esize, const SolvePlan& p, cudaStream_t s) {
+  switch (kind) {
+    case 4:
+      if (group == 64) return launch_dtype<ELEM_INT8, SCALE_BF16, 4, EXT>(L, count, esize, p, s);
+      return launch_dtype<ELEM_INT8, SCALE_BF16, 8, EXT>(L, count, esize, p, s);
+    case 5: return launch_dtype<ELEM_INT8, SCALE_E8M0, 2, EXT>(L, count, esize, p, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -52,11 +52,16 @@ typedef enum {
   DQ_ERR_UNSUPPORTED = 8    /* a shape the kernels do not handle (e.g. rows too many)    */
 } dq_status;
 
-typedef enum { DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_MXFP4 = 2, DQ_NVFP4 = 3 } dq_kind;
+typedef enum {
+  DQ_INT4 = 0, DQ_MXINT4 = 1, DQ_MXFP4 = 2, DQ_NVFP4 = 3, DQ_INT8 = 4, DQ_MXINT8 = 5
+} dq_kind;
 
 /* Format: kind plus block length along a row. INT4: group 64 or 128 (bf16 block scale,
  * elements -7..7). MXINT4: 32 (E8M0, elements -7..7). MXFP4: 32 (E8M0, E2M1 elements).
- * NVFP4: 16 (E4M3 block scale times an fp32 tensor scale, E2M1 elements). */
+ * NVFP4: 16 (E4M3 block scale times an fp32 tensor scale, E2M1 elements). The 8-bit formats
+ * of the DualQuant appendix's 8-bit table: INT8: group 128 (64 allowed), bf16 block scale,
+ * elements -127..127; MXINT8: 32 (E8M0, elements -127..127). 4-bit codes are packed two per
+ * byte (low nibble = even column), 8-bit codes one per byte (two's complement). */
 typedef struct {
   int32_t kind;
   int32_t group;
@@ -68,10 +73,11 @@ typedef enum { DQ_F32 = 0, DQ_BF16 = 1 } dq_dtype;
  *   W            [m, ldw] input weights (dtype of the call), 16-byte aligned, ldw*esize % 16 == 0
  *   r0           optional warm-start row-block scales [m, n/B] fp32 (projected on entry), or NULL
  *   c0           optional warm-start column scales [n] fp32 (finite, > 0), or NULL
- *   q_packed     out [m, n/2] uint8, the codes of the returned state
+ *   q_packed     out [m, n/2] uint8 (8-bit formats: [m, n], 16-byte aligned), the codes of
+ *                the returned state
  *   r            out [m, n/B] fp32, decoded row-block scales
  *   c            out [n] fp32, column scales
- *   block_scales out [m, n/B] codes of r (uint16 for INT4, uint8 otherwise)
+ *   block_scales out [m, n/B] codes of r (uint16 bf16 bits for INT4/INT8, uint8 otherwise)
  *   tensor_scale out [1] fp32, NVFP4 only (may be NULL for the other formats)
  *   mse_trace    out [iters+1] fp64, ||W - W_hat||^2/||W||^2 after init and each iteration */
 typedef struct {
@@ -172,7 +178,7 @@ DQ_API int64_t dq_solve_max_rows(int64_t n, dq_format fmt, int32_t dtype);
 /* Workspace (device bytes) needed by dq_act_quant. */
 DQ_API size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt);
 
-/* Activation rescale + 4-bit quantization (DualQuant Abstract: the column scales are
+/* Activation rescale + block quantization (DualQuant Abstract: the column scales are
  * per-channel activation rescalings applied before activation quantization; appendix
  * Table 6: activation SQNR with and without them). With W_hat = diag(r) Q diag(c), the
  * quantized GEMM consumes c * x, so x~ = fl32(X * c) per channel (c NULL: x~ = X). Per
@@ -180,8 +186,9 @@ DQ_API size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format 
  * s_t = amax(x~)/2688), q = RNE_E(fl32(x~ * fl32(1/d))).
  *   X            device [tokens, ldx] (dtype), 16-byte aligned, ldx*esize % 16 == 0
  *   c            device [n] fp32 or NULL
- *   x_packed     device out [tokens, n/2] uint8
- *   scales       device out [tokens, n/B] (uint16 bf16 bits for INT4, uint8 otherwise)
+ *   x_packed     device out [tokens, n/2] uint8, 4-byte aligned (8-bit formats: [tokens, n],
+ *                8-byte aligned)
+ *   scales       device out [tokens, n/B] (uint16 bf16 bits for INT4/INT8, uint8 otherwise)
  *   tensor_scale device out [1] fp32 (NVFP4; may be NULL otherwise) */
 DQ_API dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n,
                               int64_t ldx, const float* c, dq_format fmt, uint8_t* x_packed,
@@ -194,7 +201,8 @@ typedef enum {
   DQ_CODEC_E2M1 = 1,   /* RNE to E2M1, saturating at 6; code = sign<<3 | magnitude (uint8) */
   DQ_CODEC_E4M3 = 2,   /* RNE to E4M3 (FN), saturating at 448 (uint8)                      */
   DQ_CODEC_E8M0 = 3,   /* nearest power of two, tie up, clamped to 2^-127..2^127 (uint8)  */
-  DQ_CODEC_BF16 = 4    /* RNE to bfloat16 (uint16 bit pattern)                             */
+  DQ_CODEC_BF16 = 4,   /* RNE to bfloat16 (uint16 bit pattern)                             */
+  DQ_CODEC_INT8 = 5    /* RNE to -127..127, saturating; code = two's-complement byte       */
 } dq_codec;
 
 /* x: device fp32 [count]; codes: device [count] of the codec's code type. */

@@ -6,7 +6,13 @@ Tolerances (the solver's floating-point tolerance, written out here once):
   * block scales (discrete, on the admissible set): >= 99.9% identical, mismatches one
     admissible step apart;
   * column scales c: ||c_gpu - c_ora||_2 / ||c_ora||_2 <= 1e-4;
-  * normalised MSE trace: |mse_gpu - mse_ora| / mse_ora <= 1e-4 at every iteration;
+  * normalised MSE trace: |mse_gpu - mse_ora| <= max(1e-4 * mse_ora, 1e-6) at every
+    iteration. The GPU forms the trace by the expansion sum_j (S_j - 2 c_j N_j + c_j^2 D_j)
+    whose three terms are each about ||W||^2 and come from binary32 partial sums (relative
+    error up to ~35 units of 2^-24 each, worst case): its absolute error in normalised units
+    is bounded near 1e-5 and is about 1e-8 in practice, whatever the MSE. For the 4-bit
+    formats (MSE >= 1e-3) the relative bar is the binding one; the 8-bit formats (MSE
+    ~1e-4..1e-5) meet the absolute one;
   * NVFP4 tensor scale: bit-exact.
 Identical binary32 state gives identical codes (the decision is taken on the same binary32
 quotient); the residual differences come from summation order (binary32 block sums on the
@@ -23,6 +29,7 @@ CODE_MATCH = 0.999
 SCALE_MATCH = 0.999
 C_REL = 1e-4
 MSE_REL = 1e-4
+MSE_ABS = 1e-6
 
 
 def oracle_format(name_or_spec):
@@ -84,6 +91,8 @@ def compare_solve(h: dict, ora: dict, fmt, *, exact: bool = False, label: str = 
     rel = np.abs(mg - mo) / np.maximum(np.abs(mo), 1e-300)
     rel = np.where(mo == 0, np.abs(mg - mo), rel)
     rep["mse_rel_max"] = float(rel.max())
+    rep["mse_abs_max"] = float(np.abs(mg - mo).max())
+    mse_ok = bool(np.all(np.abs(mg - mo) <= np.maximum(MSE_REL * np.abs(mo), MSE_ABS)))
     if exact:
         assert same_q.all(), (label, "codes differ", int((~same_q).sum()))
         assert same_r.all(), (label, "scales differ", int((~same_r).sum()))
@@ -106,7 +115,7 @@ def compare_solve(h: dict, ora: dict, fmt, *, exact: bool = False, label: str = 
     if fmt.scale != "e4m3":
         np.testing.assert_array_equal(rg, F.decode_scale(sc_g, fmt))
     assert rep["c_rel"] <= C_REL, (label, rep)
-    assert rep["mse_rel_max"] <= MSE_REL, (label, rep)
+    assert mse_ok, (label, rep)
     return rep
 
 

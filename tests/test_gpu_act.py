@@ -1,4 +1,4 @@
-"""Parity of the CUDA activation rescale + 4-bit quantization with the oracle (B200).
+"""Parity of the CUDA activation rescale + block quantization with the oracle (B200).
 
 Every decision in this path is taken on the same binary32 values on both sides (the
 product X*c, the block maximum, fl32(a/q_max), the scale projection and fl32(x*1/d)), so
@@ -31,7 +31,7 @@ def _gpu_act(dq, X, fmt_name, c):
 
 
 def _check(h, ora, fmt):
-    codes = F.unpack_codes(h["x_packed"])
+    codes = F.unpack_codes(h["x_packed"], fmt.bits)
     np.testing.assert_array_equal(codes, ora["codes"])
     sc = h["scales"].view(np.uint16) if fmt.scale == "bf16" else h["scales"]
     np.testing.assert_array_equal(sc.astype(np.int64), ora["scale_codes"].astype(np.int64))
@@ -40,7 +40,7 @@ def _check(h, ora, fmt):
 
 
 def _decode_gpu(h, fmt):
-    codes = F.unpack_codes(h["x_packed"])
+    codes = F.unpack_codes(h["x_packed"], fmt.bits)
     q = F.decode_elem(codes, fmt)
     sc = h["scales"].view(np.uint16) if fmt.scale == "bf16" else h["scales"]
     s_t = h["tensor_scale"][0] if fmt.kind == "NVFP4" else None
@@ -50,7 +50,8 @@ def _decode_gpu(h, fmt):
     return dequant(d, q, fmt.block)
 
 
-@pytest.mark.parametrize("fmt_name", ["NVFP4", "INT4", "INT4_G64", "MXFP4", "MXINT4"])
+@pytest.mark.parametrize("fmt_name", ["NVFP4", "INT4", "INT4_G64", "MXFP4", "MXINT4", "INT8",
+                                      "INT8_G64", "MXINT8"])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_act_quant_bit_exact(dq, fmt_name, dtype):
     rng = np.random.default_rng(3)

@@ -54,6 +54,14 @@ def test_int4_encode_bit_exact(dq):
     np.testing.assert_array_equal(got, ref)
 
 
+def test_int8_encode_bit_exact(dq):
+    x = np.concatenate([_bf16_all(), _near(np.arange(-130, 130) + 0.5),
+                        np.random.default_rng(2).uniform(-140, 140, 200000).astype(np.float32)])
+    got = _run_encode(dq, x, dq.DQ_CODEC_INT8)
+    ref, _ = F.round_elem(x, F.make_format("INT8"))
+    np.testing.assert_array_equal(got, ref)
+
+
 def test_e4m3_encode_bit_exact(dq):
     mids = (F.E4M3_POS[:-1] + F.E4M3_POS[1:]) / 2
     x = np.concatenate([_bf16_all(), _near(mids), _near(F.E4M3_POS), [500.0, 1e30]])
@@ -84,11 +92,12 @@ def test_bf16_encode_bit_exact(dq):
     np.testing.assert_array_equal(got, F.bf16_nearest_bits(x))
 
 
-@pytest.mark.parametrize("codec,kind", [(1, "MXFP4"), (0, "MXINT4")])
-def test_element_decode_all_codes(dq, codec, kind):
-    codes = torch.arange(16, dtype=torch.uint8).cuda()
+@pytest.mark.parametrize("codec,kind,ncodes", [(1, "MXFP4", 16), (0, "MXINT4", 16),
+                                              (5, "MXINT8", 256)])
+def test_element_decode_all_codes(dq, codec, kind, ncodes):
+    codes = torch.arange(ncodes, dtype=torch.uint8).cuda()
     got = dq.decode(codes, codec).cpu().numpy().astype(np.float64)
-    np.testing.assert_array_equal(got, F.decode_elem(np.arange(16), F.make_format(kind)))
+    np.testing.assert_array_equal(got, F.decode_elem(np.arange(ncodes), F.make_format(kind)))
 
 
 def test_scale_decode_all_codes(dq):

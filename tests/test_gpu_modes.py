@@ -17,7 +17,7 @@ from tests._parity import compare_solve, assert_monotone, oracle_format, to_host
 
 pytestmark = pytest.mark.gpu
 
-FMTS = ["INT4", "MXINT4", "MXFP4", "NVFP4"]
+FMTS = ["INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8"]
 
 
 @pytest.fixture(scope="module")
@@ -68,7 +68,7 @@ def test_qchange_request_changes_nothing_else(dq, fmt_name):
         np.testing.assert_array_equal(traced[key], plain[key], err_msg=key)
 
 
-@pytest.mark.parametrize("fmt_name", ["MXFP4", "NVFP4", "INT4"])
+@pytest.mark.parametrize("fmt_name", ["MXFP4", "NVFP4", "INT4", "MXINT8"])
 @pytest.mark.parametrize("update", ["both", "row"])
 def test_qchange_is_the_definition_on_the_gpus_own_q(dq, fmt_name, update):
     """A solve stopped after t iterations returns Q^t, so the trace of one long solve must
@@ -82,7 +82,7 @@ def test_qchange_is_the_definition_on_the_gpus_own_q(dq, fmt_name, update):
     qs = []
     for t in range(T + 1):
         ht = _solve(dq, W, fmt_name, t, update=update)
-        qs.append(F.decode_elem(F.unpack_codes(ht["q_packed"]), fmt).astype(np.float64))
+        qs.append(F.decode_elem(F.unpack_codes(ht["q_packed"], fmt.bits), fmt).astype(np.float64))
     for t in range(2, T + 1):
         den = np.sqrt(np.sum(qs[t - 1] ** 2))
         want = np.sqrt(np.sum((qs[t] - qs[t - 1]) ** 2)) / den if den > 0 else 0.0

@@ -58,6 +58,13 @@ CASES = [
     ("NVFP4", "f32", 300, 512, 8),
     ("NVFP4", "bf16", 1, 64, 5),            # a single row
     ("MXFP4", "bf16", 2, 32, 5),            # one block column
+    # the 8-bit formats (appendix 8-bit table): INT8 G=128/64 with bf16 scales, MXINT8 G=32
+    ("INT8", "bf16", 200, 384, 8),
+    ("INT8", "f32", 130, 256, 6),
+    ("INT8_G64", "bf16", 96, 192, 8),
+    ("MXINT8", "bf16", 257, 224, 8),
+    ("MXINT8", "f32", 64, 160, 8),
+    ("MXINT8", "bf16", 3000, 128, 6),       # rows past the resident ones stream from L2
 ]
 
 
@@ -106,7 +113,7 @@ def test_config1_tile_full(dq):
     assert h["mse"][0] / h["mse"][-1] > 4.0, rep
 
 
-@pytest.mark.parametrize("fmt_name", ["INT4", "MXINT4", "MXFP4", "NVFP4"])
+@pytest.mark.parametrize("fmt_name", ["INT4", "MXINT4", "MXFP4", "NVFP4", "INT8", "MXINT8"])
 def test_iteration0_is_exact(dq, fmt_name):
     """iters = 0: single-scale RTN; every decision is on identical binary32 values."""
     W = _matrix(7, 300, 256, "bf16")
@@ -117,7 +124,8 @@ def test_iteration0_is_exact(dq, fmt_name):
     np.testing.assert_array_equal(h["r"], ora["r"])
 
 
-@pytest.mark.parametrize("fmt_name", ["INT4_G64", "MXINT4", "MXFP4", "NVFP4"])
+@pytest.mark.parametrize("fmt_name", ["INT4_G64", "MXINT4", "MXFP4", "NVFP4", "INT8_G64",
+                                      "MXINT8"])
 def test_warm_start_q_step_is_bit_exact(dq, fmt_name):
     """From the same binary32 state (r, c), the Q-step codes are identical and one further
     iteration agrees up to binary32-vs-binary64 summation."""
