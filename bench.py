@@ -69,9 +69,16 @@ def profiled_traffic_per_elem():
     return float(vals["dram_bytes_per_elem_solve"])
 
 
-def workload_name(count: int, elems: int, T: int) -> str:
-    return ("Llama-3.1-8B-shaped layer set (%d matrices, %.3e bf16 weights per GPU), NVFP4, %d "
-            "BCD iterations + activation rescale/NVFP4 quant 8192x4096" % (count, elems, T))
+def workload_name(count: int, elems: int, T: int, fmt: str = "NVFP4", update: str = "both",
+                  qchange: bool = False) -> str:
+    extra = ""
+    if update != "both":
+        extra += ", %s-scale updates only" % ("row" if update == "row" else "column")
+    if qchange:
+        extra += ", with the Q-change trace"
+    return ("Llama-3.1-8B-shaped layer set (%d matrices, %.3e bf16 weights per GPU), %s, %d "
+            "BCD iterations%s + activation rescale/%s quant 8192x4096"
+            % (count, elems, fmt, T, extra, fmt))
 
 
 def _peaks():
@@ -93,6 +100,14 @@ def parse():
                     help="solve only the first B blocks (profiling runs; not a bench value)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fmt", default="NVFP4",
+                    choices=["NVFP4", "MXFP4", "MXINT4", "INT4", "INT4_G64", "INT8", "MXINT8"],
+                    help="format of the solve and the activation quantization (default: the "
+                         "headline NVFP4 workload)")
+    ap.add_argument("--update", default="both", choices=["both", "row", "col"],
+                    help="ablation: update both scales (the method), only r or only c")
+    ap.add_argument("--qchange", action="store_true",
+                    help="also record the per-iteration Q-change trace")
     return ap.parse_args()
 
 
@@ -178,12 +193,19 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------------------- CPU oracle
-def cpu_sample_solve(W: np.ndarray, amax: float, iters: int):
+_ORACLE_FMT = {"NVFP4": ("NVFP4", 16), "MXFP4": ("MXFP4", 32), "MXINT4": ("MXINT4", 32),
+               "INT4": ("INT4", 128), "INT4_G64": ("INT4", 64), "INT8": ("INT8", 128),
+               "MXINT8": ("MXINT8", 32)}
+
+
+def cpu_sample_solve(W: np.ndarray, amax: float, iters: int, fmt: str = "NVFP4",
+                     update: str = "both"):
     """Oracle solve of a bounded sample; returns (elem*iter/s, seconds, elements)."""
     from oracle import formats as F
     from oracle import solver as S
     t0 = time.perf_counter()
-    S.solve(W, F.make_format("NVFP4"), iters, amax=amax)
+    S.solve(W, F.make_format(*_ORACLE_FMT[fmt]), iters, amax=amax if fmt == "NVFP4" else None,
+            update=update)
     dt = time.perf_counter() - t0
     return W.size * iters / dt, dt, W.size
 
@@ -230,7 +252,8 @@ def run_ours(args, world, rank, local):
     if args.blocks is not None:
         layer = [e for e in layer if e[0] < args.blocks]
     T = cfg.iters
-    fmt = dq.fmt_of(cfg.fmt)
+    fmt = dq.fmt_of(args.fmt)
+    headline = args.fmt == "NVFP4" and args.update == "both" and not args.qchange
     stream = torch.cuda.current_stream(dev)
 
     # inputs (device-generated, seeded per rank) and preallocated outputs
@@ -241,13 +264,18 @@ def run_ours(args, world, rank, local):
     ms = (ctypes.c_int64 * count)(*[W.shape[0] for W in Ws])
     ns = (ctypes.c_int64 * count)(*[W.shape[1] for W in Ws])
     lib = _lib.get()
-    ws_bytes = lib.dq_solve_workspace_bytes(count, ms, ns, fmt, T)
+    opts = None
+    if not headline and (args.update != "both" or args.qchange):
+        qtraces = [torch.empty((T + 1,), dtype=torch.float64, device=dev) for _ in Ws]
+        qptrs = (ctypes.c_void_p * count)(*[q.data_ptr() for q in qtraces]) if args.qchange \
+            else None
+        opts = _lib.dq_solve_options(dq.api.UPDATES[args.update], qptrs)
+    ws_bytes = lib.dq_solve_workspace_bytes_ex(count, ms, ns, fmt, T,
+                                               ctypes.byref(opts) if opts else None)
     ws = torch.empty((ws_bytes,), dtype=torch.uint8, device=dev)
-    act_out = dict(x_packed=torch.empty((X.shape[0], X.shape[1] // 2), dtype=torch.uint8,
-                                        device=dev),
-                   scales=torch.empty((X.shape[0], X.shape[1] // 16), dtype=torch.uint8,
-                                      device=dev),
-                   tensor_scale=torch.empty((1,), dtype=torch.float32, device=dev))
+    act_proto = dq.api.solve_outputs(X.shape[0], X.shape[1], fmt, 0, dev)
+    act_out = dict(x_packed=act_proto["q_packed"], scales=act_proto["block_scales"],
+                   tensor_scale=act_proto["tensor_scale"])
     act_ws = torch.empty((256,), dtype=torch.uint8, device=dev)
     k0 = next(i for i, (b, p, _, _) in enumerate(layer) if b == 0 and p == 1)
 
@@ -264,8 +292,13 @@ def run_ours(args, world, rank, local):
     sptr = ctypes.c_void_p(stream.cuda_stream)
 
     def step(mats_arr, Xin):
-        st = lib.dq_solve_batched(mats_arr, count, _lib.DQ_BF16, fmt, T,
-                                  ctypes.c_void_p(ws.data_ptr()), ws_bytes, sptr)
+        if opts is None:
+            st = lib.dq_solve_batched(mats_arr, count, _lib.DQ_BF16, fmt, T,
+                                      ctypes.c_void_p(ws.data_ptr()), ws_bytes, sptr)
+        else:
+            st = lib.dq_solve_batched_ex(mats_arr, count, _lib.DQ_BF16, fmt, T,
+                                         ctypes.byref(opts), ctypes.c_void_p(ws.data_ptr()),
+                                         ws_bytes, sptr)
         if st != 0:
             raise dq.DQError(st, "dq_solve_batched")
         st = lib.dq_act_quant(ctypes.c_void_p(Xin.data_ptr()), _lib.DQ_BF16, Xin.shape[0],
@@ -329,8 +362,11 @@ def run_ours(args, world, rank, local):
     alu_peak = 148 * 128 * sm_max * 1e6 / 1e12                         # Tops/s FP32
     ops = args.steps * elems * (OPS_PER_ELEM_ITER * T + OPS_PER_ELEM_INIT)
     achieved = ops / (kern_ms * 1e-3) / 1e12 if kern_ms > 0 else None
-    hbm_equiv = args.steps * elems * T * HBM_BYTES_PER_ELEM_ITER / (kern_ms * 1e-3) / 1e9
-    tpe = profiled_traffic_per_elem()
+    # W in bf16 plus the block-scale state read and written once per iteration
+    scb = 2 if args.fmt.startswith("INT") else 1
+    hbm_bpe = 2.0 + 2.0 * scb / fmt.group
+    hbm_equiv = args.steps * elems * T * hbm_bpe / (kern_ms * 1e-3) / 1e9
+    tpe = profiled_traffic_per_elem() if headline else None
     traffic = tpe * elems / per_step if tpe is not None else None        # bytes per launch
     roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tops/s",
             "frac": achieved / alu_peak if achieved else None, "traffic": traffic,
@@ -338,7 +374,7 @@ def run_ours(args, world, rank, local):
             "peak_source": "148 SMs x 128 FP32 lanes x %.0f MHz (FMA = 1 op)" % sm_max,
             "kernel": "solve_kernel", "kernel_ms_per_step": kern_ms / args.steps,
             "launches_timed": used,
-            "hbm_equivalent": {"bytes_per_elem_iter": HBM_BYTES_PER_ELEM_ITER,
+            "hbm_equivalent": {"bytes_per_elem_iter": hbm_bpe,
                                "achieved_GBps": hbm_equiv,
                                "frac_of_hbm_peak": hbm_equiv / float(peaks["hbm_gbs"]),
                                "peak_GBps": float(peaks["hbm_gbs"]), "peak_source": peak_src}}
@@ -353,10 +389,10 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         Wk = Ws[k0].float().cpu().numpy().astype(np.float64)
         amax = float(np.max(np.abs(Wk)))
-        v, dt, n_el = cpu_sample_solve(Wk, amax, T)
+        v, dt, n_el = cpu_sample_solve(Wk, amax, T, args.fmt, args.update)
         cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "block-0 k_proj (1024x4096) of this layer set, 16 iterations, "
-                         "%.1f s, single process" % dt}
+               "sample": "block-0 k_proj (1024x4096) of this layer set, %s, 16 iterations, "
+                         "%.1f s, single process" % (args.fmt, dt)}
 
     if rank == 0:
         line = {
@@ -364,7 +400,8 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": workload_name(count, elems, T),
+            "config": {"workload": workload_name(count, elems, T, args.fmt, args.update,
+                                                 args.qchange),
                        "full_model_solve_s": ms_step * 1e-3,
                        "l2": "inputs larger than L2 (%.1f GB of weights per step)"
                              % (elems * 2 / 1e9),
