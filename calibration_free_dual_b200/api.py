@@ -209,6 +209,25 @@ def act_quant(X: torch.Tensor, fmt, c: torch.Tensor | None = None, stream=None) 
     return o
 
 
+def w4a4_gemm(x: dict, w: dict, fmt="NVFP4", stream=None) -> torch.Tensor:
+    """dq_w4a4_gemm: y[T, N] from act_quant's output `x` (x_packed, scales, tensor_scale)
+    and a solve's output `w` (q_packed, block_scales, tensor_scale)."""
+    f = fmt_of(fmt)
+    xq, xs, xst = x["x_packed"], x["scales"], x["tensor_scale"]
+    wq, ws, wst = w["q_packed"], w["block_scales"], w["tensor_scale"]
+    for t, name in ((xq, "x_packed"), (xs, "scales"), (wq, "q_packed"), (ws, "block_scales")):
+        _need_cuda(t, name)
+        if not t.is_contiguous():
+            raise ValueError(name + " must be contiguous")
+    T, N, K = xq.shape[0], wq.shape[0], xq.shape[1] * 2
+    if wq.shape[1] * 2 != K:
+        raise ValueError("activation and weight K differ")
+    y = torch.empty((T, N), dtype=torch.float32, device=xq.device)
+    _check(_lib.get().dq_w4a4_gemm(_p(xq), _p(xs), _p(xst), T, _p(wq), _p(ws), _p(wst), N, K, f,
+                                   _p(y), N, _stream_ptr(stream)), "dq_w4a4_gemm")
+    return y
+
+
 _CODE_DTYPE = {_lib.DQ_CODEC_BF16: torch.int16}
 
 

@@ -305,6 +305,42 @@ dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, int64_t l
   return dq_solve_batched(&d, 1, dtype, fmt, iters, workspace, workspace_bytes, stream);
 }
 
+dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
+                       const float* x_tensor_scale, int64_t T, const uint8_t* w_packed,
+                       const uint8_t* w_scales, const float* w_tensor_scale, int64_t N,
+                       int64_t K, dq_format fmt, float* y, int64_t ldy, void* stream) {
+  dq_status st = check_format(fmt);
+  if (st != DQ_OK) return st;
+  if (fmt.kind != DQ_NVFP4) return DQ_ERR_UNSUPPORTED;
+  if (T <= 0 || N <= 0 || K <= 0 || ldy < N) return DQ_ERR_INVALID_ARG;
+  if (K % 64 != 0) return DQ_ERR_SHAPE;
+  if (T > ((int64_t)1 << 30) || N > ((int64_t)1 << 30) || K > ((int64_t)1 << 30))
+    return DQ_ERR_SHAPE;
+  if (x_packed == nullptr || x_scales == nullptr || x_tensor_scale == nullptr ||
+      w_packed == nullptr || w_scales == nullptr || w_tensor_scale == nullptr || y == nullptr)
+    return DQ_ERR_INVALID_ARG;
+  if (!aligned16(x_packed) || !aligned16(w_packed)) return DQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x_scales) & 3u) || (reinterpret_cast<uintptr_t>(w_scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(y) & 3u))
+    return DQ_ERR_INVALID_ARG;
+  unsigned* errp = nullptr;
+  if ((st = err_word_ptr(&errp)) != DQ_OK) return st;
+  dq::GemmArgs A;
+  A.xq = x_packed;
+  A.xs = x_scales;
+  A.xst = x_tensor_scale;
+  A.wq = w_packed;
+  A.ws = w_scales;
+  A.wst = w_tensor_scale;
+  A.y = y;
+  A.T = T;
+  A.N = N;
+  A.K = K;
+  A.ldy = ldy;
+  A.err_word = errp;
+  return from_cuda(dq::launch_w4a4_gemm(A, static_cast<cudaStream_t>(stream)));
+}
+
 size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt) {
   if (tokens < 0 || n <= 0 || check_format(fmt) != DQ_OK) return 0;
   return 256;

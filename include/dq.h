@@ -195,6 +195,28 @@ DQ_API dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int6
                               void* scales, float* tensor_scale, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* W4A4 GEMM on the quantized operands: the deployment side of the dual-scale model (the
+ * ai4snews summary of DualQuant, paragraph 4: a real packed W4A4 inference path). With
+ * W_hat = diag(r) Q diag(c) and the activation x~ = c * x quantized per (token, block) as
+ * d * q_x, the layer output is
+ *   y[t, i] = sum_j (d q_x)[t, j] * (r q)[i, j]
+ * computed on the tensor cores (block-scaled FP4 MMA, fp32 accumulation). NVFP4 only:
+ * E2M1 elements, E4M3 block scales per 16 elements, one fp32 tensor scale per operand.
+ *   x_packed        device [T, K/2] uint8 (dq_act_quant's x_packed), 16-byte aligned
+ *   x_scales        device [T, K/16] uint8 (its scales; code 0 = an all-zero block), 4-byte
+ *                   aligned
+ *   x_tensor_scale  device [1] fp32
+ *   w_packed        device [N, K/2] uint8 (dq_solve's q_packed), 16-byte aligned
+ *   w_scales        device [N, K/16] uint8 (its block_scales), 4-byte aligned
+ *   w_tensor_scale  device [1] fp32 (its tensor_scale)
+ *   y               device out [T, ldy] fp32, ldy >= N
+ * Returns DQ_ERR_SHAPE if K is not a multiple of 64, DQ_ERR_UNSUPPORTED for another format;
+ * a bounded wait that gives up raises DQ_ERR_TIMEOUT in the device error word. */
+DQ_API dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
+                              const float* x_tensor_scale, int64_t T, const uint8_t* w_packed,
+                              const uint8_t* w_scales, const float* w_tensor_scale, int64_t N,
+                              int64_t K, dq_format fmt, float* y, int64_t ldy, void* stream);
+
 /* Codecs used by the kernels, exposed for bit-exact tests (one code per output element). */
 typedef enum {
   DQ_CODEC_INT4 = 0,   /* RNE to -7..7, saturating; code = two's-complement nibble (uint8) */

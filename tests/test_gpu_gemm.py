@@ -1,0 +1,104 @@
+"""The W4A4 GEMM on the tensor cores against the oracle's plain definition (B200).
+
+Operands are the 4-bit codes and E4M3 block-scale codes the solver and the activation
+quantizer produce. The tensor core accumulates in binary32, 64 elements per instruction, so
+the bar is |y - y_oracle| <= (K/64 + 4) * 2^-23 * sum_j |x_hat w_hat| (one binary32
+rounding per instruction and a few for the final scaling), elementwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats as F
+from oracle import gemm as G
+from oracle import solver as S
+
+pytestmark = pytest.mark.gpu
+NV = F.make_format("NVFP4")
+
+
+@pytest.fixture(scope="module")
+def dq():
+    import calibration_free_dual_b200 as pkg
+    return pkg
+
+
+def _operand(rng, rows, K, zero_frac=0.0):
+    codes = rng.integers(0, 16, (rows, K)).astype(np.uint8)
+    sc = rng.integers(1, 127, (rows, K // 16)).astype(np.uint8)
+    if zero_frac:
+        z = rng.random((rows, K // 16)) < zero_frac
+        sc[z] = 0
+        codes[np.repeat(z, 16, axis=1)] = 0
+    return codes, sc
+
+
+def _gpu(dq, xc, xs, sx, wc, ws, sw):
+    dev = torch.device("cuda")
+    x = dict(x_packed=torch.from_numpy(F.pack_codes(xc)).to(dev),
+             scales=torch.from_numpy(xs).to(dev),
+             tensor_scale=torch.tensor([sx], dtype=torch.float32, device=dev))
+    w = dict(q_packed=torch.from_numpy(F.pack_codes(wc)).to(dev),
+             block_scales=torch.from_numpy(ws).to(dev),
+             tensor_scale=torch.tensor([sw], dtype=torch.float32, device=dev))
+    y = dq.w4a4_gemm(x, w)
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    return y.cpu().numpy().astype(np.float64)
+
+
+def _check(y, xc, xs, sx, wc, ws, sw, K):
+    ref = G.w4a4_gemm(xc, xs, sx, wc, ws, sw, NV)
+    bound = (K / 64 + 4) * 2.0 ** -23 * G.abs_products(xc, xs, sx, wc, ws, sw, NV) + 1e-30
+    err = np.abs(y - ref)
+    assert np.all(err <= bound), (float((err / bound).max()), np.argwhere(err > bound)[:5])
+
+
+@pytest.mark.parametrize("T,N,K", [(128, 128, 256), (256, 384, 1024), (200, 136, 320),
+                                   (1, 8, 64), (130, 260, 4096)])
+def test_gemm_matches_oracle(dq, T, N, K):
+    rng = np.random.default_rng(T * 7 + N + K)
+    xc, xs = _operand(rng, T, K, zero_frac=0.05)
+    wc, ws = _operand(rng, N, K)
+    sx, sw = np.float32(0.03125), np.float32(0.0017)
+    y = _gpu(dq, xc, xs, sx, wc, ws, sw)
+    _check(y, xc, xs, sx, wc, ws, sw, K)
+
+
+def test_gemm_on_the_solver_and_activation_outputs(dq):
+    """Solve a weight in NVFP4, quantize an activation with its column scales, multiply:
+    matches the oracle GEMM of the same codes, and approximates W x."""
+    rng = np.random.default_rng(9)
+    m, K, T = 384, 1024, 130
+    w = rng.standard_t(4, (m, K)) * 0.014
+    w[:, rng.choice(K, 4, replace=False)] *= 10.0
+    W = torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16).cuda()
+    sol = dq.solve(W, "NVFP4", 8)
+    X = rng.standard_normal((T, K)).astype(np.float32)
+    X[:, rng.choice(K, 6, replace=False)] *= 50.0
+    X[3] = 0.0
+    Xt = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    act = dq.act_quant(Xt, "NVFP4", sol["c"])
+    y = dq.w4a4_gemm(act, sol)
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    y = y.cpu().numpy().astype(np.float64)
+    xc = F.unpack_codes(act["x_packed"].cpu().numpy())
+    xs = act["scales"].cpu().numpy()
+    sx = act["tensor_scale"].cpu().numpy()[0]
+    wc = F.unpack_codes(sol["q_packed"].cpu().numpy())
+    ws = sol["block_scales"].cpu().numpy()
+    sw = sol["tensor_scale"].cpu().numpy()[0]
+    _check(y, xc, xs, sx, wc, ws, sw, K)
+    assert np.all(y[3] == 0.0)
+    ref = Xt.float().cpu().numpy().astype(np.float64) @ W.float().cpu().numpy().astype(np.float64).T
+    rel = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert rel < 0.2, rel                      # 4-bit weights and activations
+
+
+def test_gemm_rejects_bad_shapes(dq):
+    f = dq.fmt_of("NVFP4")
+    nul = None
+    assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 96, f, nul, 8, nul) == 2
+    assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 128, dq.fmt_of("MXFP4"), nul, 8,
+                           nul) == 8
