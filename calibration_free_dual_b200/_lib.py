@@ -57,9 +57,10 @@ SIGNATURES = {
     "dq_act_quant": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, c_void_p,
                                dq_format, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
+    "dq_w4a4_gemm_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int64]),
     "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                c_void_p, c_int64, c_int64, dq_format, c_void_p, c_int64,
-                               c_void_p]),
+                               c_void_p, c_size_t, c_void_p]),
     "dq_encode": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p]),
     "dq_decode": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p]),
     "dq_last_device_error": (c_int32, [c_void_p]),

@@ -209,7 +209,8 @@ def act_quant(X: torch.Tensor, fmt, c: torch.Tensor | None = None, stream=None) 
     return o
 
 
-def w4a4_gemm(x: dict, w: dict, fmt="NVFP4", stream=None) -> torch.Tensor:
+def w4a4_gemm(x: dict, w: dict, fmt="NVFP4", stream=None,
+              workspace: torch.Tensor | None = None) -> torch.Tensor:
     """dq_w4a4_gemm: y[T, N] from act_quant's output `x` (x_packed, scales, tensor_scale)
     and a solve's output `w` (q_packed, block_scales, tensor_scale)."""
     f = fmt_of(fmt)
@@ -223,8 +224,15 @@ def w4a4_gemm(x: dict, w: dict, fmt="NVFP4", stream=None) -> torch.Tensor:
     if wq.shape[1] * 2 != K:
         raise ValueError("activation and weight K differ")
     y = torch.empty((T, N), dtype=torch.float32, device=xq.device)
-    _check(_lib.get().dq_w4a4_gemm(_p(xq), _p(xs), _p(xst), T, _p(wq), _p(ws), _p(wst), N, K, f,
-                                   _p(y), N, _stream_ptr(stream)), "dq_w4a4_gemm")
+    lib = _lib.get()
+    need = lib.dq_w4a4_gemm_workspace_bytes(T, N, K)
+    if need == 0:
+        raise DQError(_lib.DQ_ERR_SHAPE, "K must be a multiple of 64")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=xq.device)
+    _check(lib.dq_w4a4_gemm(_p(xq), _p(xs), _p(xst), T, _p(wq), _p(ws), _p(wst), N, K, f,
+                            _p(y), N, _p(workspace), need, _stream_ptr(stream)),
+           "dq_w4a4_gemm")
     return y
 
 

@@ -305,10 +305,16 @@ dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, int64_t l
   return dq_solve_batched(&d, 1, dtype, fmt, iters, workspace, workspace_bytes, stream);
 }
 
+size_t dq_w4a4_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K) {
+  if (T <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return dq::gemm_workspace_bytes(T, N, K);
+}
+
 dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
                        const float* x_tensor_scale, int64_t T, const uint8_t* w_packed,
                        const uint8_t* w_scales, const float* w_tensor_scale, int64_t N,
-                       int64_t K, dq_format fmt, float* y, int64_t ldy, void* stream) {
+                       int64_t K, dq_format fmt, float* y, int64_t ldy, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   dq_status st = check_format(fmt);
   if (st != DQ_OK) return st;
   if (fmt.kind != DQ_NVFP4) return DQ_ERR_UNSUPPORTED;
@@ -323,6 +329,9 @@ dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
   if ((reinterpret_cast<uintptr_t>(x_scales) & 3u) || (reinterpret_cast<uintptr_t>(w_scales) & 3u) ||
       (reinterpret_cast<uintptr_t>(y) & 3u))
     return DQ_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < dq_w4a4_gemm_workspace_bytes(T, N, K))
+    return DQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DQ_ERR_INVALID_ARG;
   unsigned* errp = nullptr;
   if ((st = err_word_ptr(&errp)) != DQ_OK) return st;
   dq::GemmArgs A;
@@ -338,7 +347,7 @@ dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
   A.K = K;
   A.ldy = ldy;
   A.err_word = errp;
-  return from_cuda(dq::launch_w4a4_gemm(A, static_cast<cudaStream_t>(stream)));
+  return from_cuda(dq::launch_w4a4_gemm(A, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt) {

@@ -4,17 +4,23 @@
 // summary, paragraph 4: a real packed W4A4 inference path); the column scale c has already
 // moved into the activation (dq_act_quant), so the GEMM sees two block-scaled operands.
 //
-// sm_100a design: 5th-generation tensor cores, block-scaled. One CTA (128 threads) owns a
-// 128 x 128 output tile, accumulated in tensor memory (TMEM) by
-// tcgen05.mma.kind::mxf4nvf4.block_scale (M = 128, N = 128, K = 64 per instruction), issued by
-// one thread. The K loop is double-buffered: all threads stage the next 256-wide K slice of
-// both operands into shared memory (cp.async, canonical K-major no-swizzle core-matrix layout)
-// and its scale factors in the 128 x 4 interleaved layout the tensor core reads, while the
-// tensor core works on the current slice; the scale factors go to TMEM with tcgen05.cp. The
-// epilogue reads the accumulator with tcgen05.ld, multiplies by the two tensor scales and
-// stores fp32. Every wait on an mbarrier is bounded: on timeout the kernel raises the error
-// word, drains its own copies, frees its TMEM and returns.
+// sm_100a design: 5th-generation tensor cores, block-scaled, warp-specialized. One CTA (six
+// warps, one per SM) owns a 128 x 256 output tile accumulated in tensor memory (TMEM) by
+// tcgen05.mma.kind::mxf4nvf4.block_scale (M = 128, N = 256, K = 64 per instruction):
+//   * warp 0 (one lane) produces: per 256-wide K slice, two TMA tile loads (128-byte
+//     swizzle) of the packed E2M1 codes and three bulk copies of the scale factors, all
+//     completing on the slice's "full" mbarrier; four slices in flight;
+//   * warp 1 (one lane) consumes: copies the slice's scale factors to TMEM (tcgen05.cp),
+//     issues the four MMAs and commits them to the slice's "empty" mbarrier;
+//   * warps 2-5 wait for the last commit, read the accumulator (tcgen05.ld), apply the two
+//     tensor scales and store fp32.
+// The scale factors are first re-laid (a small pre-pass per operand) into the 128-row x 4
+// interleaving the tensor core reads, so a slice's scale factors are one contiguous copy.
+// Every mbarrier wait is bounded by the global timer; on timeout the kernel raises the error
+// word, frees its TMEM and returns.
+#include <algorithm>
 #include <cstdint>
+#include <cuda.h>   // CUtensorMap and its enums (the encoder is fetched from the driver)
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
@@ -22,41 +28,52 @@
 namespace dq {
 namespace {
 
-constexpr int GT = 128;                 // threads per CTA
-constexpr int BM = 128, BN = 128;       // output tile (tokens x weight rows)
-constexpr int BKE = 256;                // K elements per stage (4 MMAs of K = 64)
-constexpr int BKB = BKE / 2;            // bytes of packed E2M1 per row per stage
-constexpr int STAGES = 2;
-constexpr int OP_BYTES = BM * BKB;      // one operand's stage: 16 KB
-constexpr int SF_BYTES = BM * BKE / 16; // one operand's scale factors per stage: 2 KB
-constexpr int STAGE_BYTES = 2 * OP_BYTES + 2 * SF_BYTES;
+constexpr int GT = 192;                 // threads per CTA: producer, MMA, 4 epilogue warps
+constexpr int BM = 128, BN = 256;       // output tile (tokens x weight rows)
+constexpr int BKE = 256;                // K elements per slice (4 MMAs of K = 64)
+constexpr int BKB = BKE / 2;            // bytes of packed E2M1 per row per slice (128)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BKB;       // 16 KB
+constexpr int B_BYTES = BN * BKB;       // 32 KB
+constexpr int SFA_BYTES = BM * BKE / 16;   // 2 KB: 4 blocks of 512 (one per MMA)
+constexpr int SFB_BYTES = BN * BKE / 16;   // 4 KB: 2 row halves x 4 blocks of 512
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = 80 * 1024;   // > 1/3 of the SM: at most two CTAs (and 2 x 256 TMEM
-                                        // columns) per SM, so a TMEM allocation never waits
-constexpr uint32_t TMEM_COLS = 256;     // accumulator 128 + scale factors 2 x (16 + 16)
-constexpr uint32_t SFA_COL = 128, SFB_COL = 160;   // + 16 per buffer
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s: far beyond any stage's work
+constexpr int SMEM_BYTES = BAR_OFF + 128 + 1024;   // barriers, TMEM slot, 1024-byte alignment
+constexpr uint32_t TMEM_COLS = 512;     // accumulator 256 + scale factors 4 x (16 + 32)
+constexpr uint32_t SF_COL0 = 256, SF_COLS_PER_STAGE = 48;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s: far beyond any slice's work
 
-static_assert(BAR_OFF + 64 <= SMEM_BYTES, "shared memory layout");
+static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned slices (128-byte swizzle)");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+static_assert(SF_COL0 + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// ---- cp.async (16 bytes, L2 only; 4 bytes) with zero fill when src_size is 0
-__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t src_size) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_size));
+// ---- TMA tile loads and bulk copies, completing on an mbarrier (byte count)
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
-__device__ __forceinline__ void cp4(uint32_t dst, const void* src, uint32_t src_size) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(src_size));
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N)); }
 
 // ---- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes)
+               : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -99,17 +116,23 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// shared-memory matrix descriptor: no swizzle, K-major canonical layout of 8-row x 16-byte
-// core matrices; lbo = byte distance between the two 16-byte K halves an MMA reads, sbo =
-// byte distance between consecutive groups of 8 rows; version 1 (sm_100)
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// shared-memory matrix descriptor (sm_100 version 1): start address, leading and stride
+// byte offsets, layout type (0: no swizzle, 2: 128-byte swizzle)
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(layout & 7u) << 61;
   return d;
 }
+// K-major operand slice written by a 128-byte-swizzled TMA box of 128-byte rows: 8-row
+// groups 1024 bytes apart; an MMA's K = 64 slice starts 32 bytes further per step
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr) { return smem_desc(addr, 16, 1024, 2); }
+// scale factors: 32 rows x 16 bytes, 8-row groups 128 bytes apart, no swizzle
+__device__ __forceinline__ uint64_t sf_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
 // 32 rows x 128 bits of scale factors from shared memory to TMEM, replicated into the four
 // 32-lane sub-partitions
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
@@ -149,167 +172,214 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// instruction descriptor: A, B E2M1 (1), scale factors UE4M3 (0), K-major, M = 128, N = 128
+
+// instruction descriptor: A, B E2M1 (1), scale factors UE4M3 (0), K-major, M = 128, N = 256
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(BM >> 4) << 24);
 
-// One stage of loads: the 256-wide K slice [k0, k0 + 256) of the 128 rows [row0, row0 + 128)
-// of one operand (codes [rows, K/2] bytes, scale codes [rows, K/16] bytes).
-//   codes -> smem offset kc*2048 + (row/8)*128 + (row%8)*16 for the 16-byte chunk kc (32
-//            elements): MMA kb reads chunks 2kb, 2kb+1 (lbo 2048, sbo 128);
-//   scale codes -> the 512-byte block of MMA kb, byte (row%32)*16 + (row/32)*4 + s for its
-//            s-th scale (s < 4): the 128 x 4 interleaving tcgen05.cp 32x128b.warpx4 expects.
-// Rows past `rows` and columns past K are zero-filled (scale 0 = no contribution).
-__device__ __forceinline__ void load_stage(const uint8_t* codes, const uint8_t* scales,
-                                           int64_t rows, int64_t K, int64_t row0, int64_t k0,
-                                           uint32_t s_codes, uint32_t s_sf, int tid) {
-  const int64_t kbytes = K / 2, kscales = K / 16;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = tid + GT * i;                    // 1024 chunks: 8 rows x 8 chunks x 16 groups
-    const int r8 = c & 7, kc = (c >> 3) & 7, rg = c >> 6;
-    const int row = rg * 8 + r8;
-    const int64_t grow = row0 + row;
-    const bool ok = grow < rows && k0 + 32 * kc < K;
-    const uint8_t* src = ok ? codes + grow * kbytes + k0 / 2 + 16 * kc : codes;
-    cp16(s_codes + kc * 2048 + rg * 128 + r8 * 16, src, ok ? 16u : 0u);
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = tid + GT * i;                    // 512 groups of 4 scales: 128 rows x 4 MMAs
-    const int row = c & 127, kb = c >> 7;
-    const int64_t grow = row0 + row;
-    const bool ok = grow < rows && k0 + 64 * kb < K;
-    const uint8_t* src = ok ? scales + grow * kscales + k0 / 16 + 4 * kb : scales;
-    cp4(s_sf + kb * 512 + (row & 31) * 16 + (row >> 5) * 4, src, ok ? 4u : 0u);
+// Scale codes [rows, K/16] -> [row block of 128][K/64][512 bytes]: in each 512-byte block the
+// four scales of row r of the block (for one MMA's 64 elements) sit at (r % 32) * 16 +
+// (r / 32) * 4, the layout tcgen05.cp 32x128b.warpx4 expects. Rows in [rows, rows_pad) are 0.
+__global__ void sf_interleave_kernel(const uint8_t* __restrict__ src, int64_t rows,
+                                     int64_t rows_pad, int64_t K, uint8_t* __restrict__ dst) {
+  const int64_t kq = K / 64;
+  const int64_t total = rows_pad * kq;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / kq, g = i % kq;
+    uint32_t v = 0u;
+    if (row < rows) v = *reinterpret_cast<const uint32_t*>(src + row * (K / 16) + 4 * g);
+    const int r = (int)(row & 127);
+    uint8_t* blk = dst + ((row >> 7) * kq + g) * 512;
+    *reinterpret_cast<uint32_t*>(blk + (r & 31) * 16 + (r >> 5) * 4) = v;
   }
 }
 
-__global__ void __launch_bounds__(GT, 1) w4a4_gemm_kernel(const __grid_constant__ GemmArgs A) {
-  extern __shared__ __align__(1024) unsigned char smem[];
+__global__ void __launch_bounds__(GT, 1)
+w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ GemmArgs A) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.y * BM, n0 = (int64_t)blockIdx.x * BN;
-  const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + BAR_OFF;           // mbar[0], mbar[1]: MMAs of a stage done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BAR_OFF + 16);
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;               // 1024-byte aligned slices
+  unsigned char* base_ptr = smem_raw + (sbase - raw);
+  const uint32_t full0 = sbase + BAR_OFF;                      // full[s]  = full0 + 8s
+  const uint32_t empty0 = full0 + 8 * STAGES;                  // empty[s] = empty0 + 8s
+  const uint32_t accbar = empty0 + 8 * STAGES;                 // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BAR_OFF + 8 * (2 * STAGES + 1));
+  volatile int* fail = reinterpret_cast<volatile int*>(base_ptr + BAR_OFF + 8 * (2 * STAGES + 2));
 
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-  if (tid == 0) {
-    mbar_init(bar0, 1);
-    mbar_init(bar0 + 8, 1);
+  if (tid == 32) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(accbar, 1);
+    *fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   const int nk = (int)((A.K + BKE - 1) / BKE);
-  uint32_t phase[STAGES] = {0u, 0u};
-  bool timeout = false;
+  const int64_t kq = A.K / 64;
 
-  auto stage_addr = [&](int buf) { return sbase + buf * STAGE_BYTES; };
-  auto issue = [&](int k, int buf) {
-    const uint32_t s = stage_addr(buf);
-    load_stage(A.xq, A.xs, A.T, A.K, t0, (int64_t)k * BKE, s, s + 2 * OP_BYTES, tid);
-    load_stage(A.wq, A.ws, A.N, A.K, n0, (int64_t)k * BKE, s + OP_BYTES,
-               s + 2 * OP_BYTES + SF_BYTES, tid);
-    cp_commit();
-  };
-
-  issue(0, 0);
-  for (int k = 0; k < nk && !timeout; ++k) {
-    const int buf = k & 1;
-    if (k + 1 < nk) {
-      if (k >= 1) {
-        // the MMAs of stage k-1 read buffer (k+1)&1: thread 0 waits for them (bounded), the
-        // barrier makes the outcome uniform before anyone refills the buffer
-        const int pb = (k + 1) & 1;
-        const bool ok = tid != 0 || mbar_wait(bar0 + 8 * pb, phase[pb]);
-        phase[pb] ^= 1u;
-        timeout = __syncthreads_or(!ok) != 0;
-      }
-      if (timeout) break;
-      issue(k + 1, (k + 1) & 1);
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
+  if (warp == 0 && lane == 0) {
+    // ---- producer
+    for (int k = 0; k < nk; ++k) {
+      const int s = k % STAGES;
+      const uint32_t use = (uint32_t)(k / STAGES);             // how often slot s was used
+      if (!mbar_wait(empty0 + 8 * s, (use & 1u) ^ 1u)) { *fail = 1; break; }
+      if (*fail) break;
+      const int nkb = (int)((kq - 4ll * k) < 4 ? (kq - 4ll * k) : 4);
+      const uint32_t sf_bytes = 512u * nkb;
+      const uint32_t st = sbase + s * STAGE_BYTES;
+      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES + 3 * sf_bytes);
+      tma_load_2d(st, &tmA, k * BKB, (int)t0, full0 + 8 * s);
+      tma_load_2d(st + A_BYTES, &tmB, k * BKB, (int)n0, full0 + 8 * s);
+      bulk_load(st + A_BYTES + B_BYTES, A.sfa + ((t0 >> 7) * kq + 4ll * k) * 512, sf_bytes,
+                full0 + 8 * s);
+      bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, A.sfb + ((n0 >> 7) * kq + 4ll * k) * 512,
+                sf_bytes, full0 + 8 * s);
+      bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + 2048,
+                A.sfb + (((n0 >> 7) + 1) * kq + 4ll * k) * 512, sf_bytes, full0 + 8 * s);
     }
-    fence_async_smem();              // this thread's copies, visible to the tensor core
-    __syncthreads();
-    if (tid == 0) {
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issue
+    bool ok = true;
+    for (int k = 0; k < nk; ++k) {
+      const int s = k % STAGES;
+      const uint32_t use = (uint32_t)(k / STAGES);
+      if (!mbar_wait(full0 + 8 * s, use & 1u) || *fail) { *fail = 1; ok = false; break; }
       tc_fence_after();
-      const uint32_t s = stage_addr(buf);
-      const int64_t left = (A.K - (int64_t)k * BKE + 63) / 64;
-      const int nkb = left < 4 ? (int)left : 4;
-      const uint32_t tsfa = tmem + SFA_COL + 16 * buf, tsfb = tmem + SFB_COL + 16 * buf;
+      const int nkb = (int)((kq - 4ll * k) < 4 ? (kq - 4ll * k) : 4);
+      const uint32_t st = sbase + s * STAGE_BYTES;
+      const uint32_t tsf = tmem + SF_COL0 + SF_COLS_PER_STAGE * s;   // SFA: +4kb, SFB: +16+8kb
       for (int kb = 0; kb < nkb; ++kb) {
-        tmem_cp_sf(tsfa + 4 * kb, smem_desc(s + 2 * OP_BYTES + kb * 512, 0, 128));
-        tmem_cp_sf(tsfb + 4 * kb, smem_desc(s + 2 * OP_BYTES + SF_BYTES + kb * 512, 0, 128));
+        tmem_cp_sf(tsf + 4 * kb, sf_desc(st + A_BYTES + B_BYTES + kb * 512));
+        tmem_cp_sf(tsf + 16 + 8 * kb, sf_desc(st + A_BYTES + B_BYTES + SFA_BYTES + kb * 512));
+        tmem_cp_sf(tsf + 16 + 8 * kb + 4,
+                   sf_desc(st + A_BYTES + B_BYTES + SFA_BYTES + 2048 + kb * 512));
       }
-      for (int kb = 0; kb < nkb; ++kb) {
-        const uint64_t ad = smem_desc(s + 2 * kb * 2048, 2048, 128);
-        const uint64_t bd = smem_desc(s + OP_BYTES + 2 * kb * 2048, 2048, 128);
-        mma_nvfp4(tmem, ad, bd, IDESC_NVFP4, (k > 0 || kb > 0) ? 1u : 0u, tsfa + 4 * kb,
-                  tsfb + 4 * kb);
-      }
-      mma_commit(bar0 + 8 * buf);
+      for (int kb = 0; kb < nkb; ++kb)
+        mma_nvfp4(tmem, operand_desc(st + 32 * kb), operand_desc(st + A_BYTES + 32 * kb),
+                  IDESC_NVFP4, (k > 0 || kb > 0) ? 1u : 0u, tsf + 4 * kb, tsf + 16 + 8 * kb);
+      mma_commit(empty0 + 8 * s);
     }
-  }
-
-  // the last stage's MMAs (in issue order after every earlier one); the outcome is made
-  // uniform across the CTA before the epilogue's warp-collective TMEM loads
-  if (!timeout && nk > 0) {
-    const int lb = (nk - 1) & 1;
-    const bool ok = tid != 0 || mbar_wait(bar0 + 8 * lb, phase[lb]);
-    timeout = __syncthreads_or(!ok) != 0;
-  }
-  cp_wait<0>();                      // no copy of ours is still in flight
-  if (timeout) {
-    if (tid == 0) atomicOr(A.err_word, ERRBIT_TIMEOUT);
-  } else {
-    tc_fence_after();
-    const float scale = __fmul_rn(*A.xst, *A.wst);
-    const int64_t t = t0 + warp * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    if (ok) mma_commit(accbar);
+  } else if (warp >= 2) {
+    // ---- epilogue: TMEM sub-partition warp % 4 holds rows 32 * (warp % 4) ...
+    const int sp = warp & 3;
+    bool ok = false;
+    if (lane == 0) ok = mbar_wait(accbar, 0) && !*fail;
+    ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+    if (ok) {
+      tc_fence_after();
+      const float scale = __fmul_rn(*A.xst, *A.wst);
+      const int64_t t = t0 + sp * 32 + lane;
+      const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        float v[32];
+        tmem_ld32(lane_addr + cb * 32, v);
+        if (t < A.T) {
+          float* yrow = A.y + t * A.ldy + n0 + cb * 32;
+          const int64_t rem = A.N - n0 - cb * 32;
+          const int64_t ncols = rem < 32 ? rem : 32;
+          if (ncols == 32 && (reinterpret_cast<uintptr_t>(yrow) & 15u) == 0) {
 #pragma unroll
-    for (int cb = 0; cb < BN / 32; ++cb) {
-      float v[32];
-      tmem_ld32(lane_addr + cb * 32, v);
-      if (t < A.T) {
-        float* yrow = A.y + t * A.ldy + n0 + cb * 32;
-        const int64_t rem = A.N - n0 - cb * 32;
-        const int64_t ncols = rem < 32 ? rem : 32;
-        if (ncols == 32 && (reinterpret_cast<uintptr_t>(yrow) & 15u) == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(yrow + i) =
-                make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
-        } else {
-          for (int i = 0; i < ncols; ++i) yrow[i] = v[i] * scale;
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(yrow + i) =
+                  make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
+          } else {
+            for (int i = 0; i < ncols; ++i) yrow[i] = v[i] * scale;
+          }
         }
       }
+    } else if (lane == 0) {
+      *fail = 1;
     }
   }
+
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && *fail) atomicOr(A.err_word, ERRBIT_TIMEOUT);
   if (warp == 0) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
+// cuTensorMapEncodeTiled from the driver (no link dependency on libcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// [rows, K/2] bytes, box of box_rows rows x 128 bytes, 128-byte swizzle, zero fill outside
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K,
+                    uint32_t box_rows) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)BKB, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
 }  // namespace
 
-size_t gemm_smem_bytes() { return SMEM_BYTES; }
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K) {
+  // interleaved scale factors: activation rows padded to 128, weight rows to 256
+  return (size_t)(round_up(T, BM) + round_up(N, BN)) * (size_t)(K / 16) + 256;
+}
 
-cudaError_t launch_w4a4_gemm(const GemmArgs& A, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(w4a4_gemm_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+cudaError_t launch_w4a4_gemm(const GemmArgs& A0, void* workspace, cudaStream_t s) {
+  GemmArgs A = A0;
+  const int64_t tpad = round_up(A.T, BM), npad = round_up(A.N, BN);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  A.sfa = ws;
+  A.sfb = ws + tpad * (A.K / 16);
+  // re-lay both operands' scale factors
+  const int64_t work_a = tpad * (A.K / 64), work_b = npad * (A.K / 64);
+  const int ga = (int)std::min<int64_t>((work_a + 255) / 256, 148 * 8);
+  const int gb = (int)std::min<int64_t>((work_b + 255) / 256, 148 * 8);
+  sf_interleave_kernel<<<ga, 256, 0, s>>>(A.xs, A.T, tpad, A.K, const_cast<uint8_t*>(A.sfa));
+  sf_interleave_kernel<<<gb, 256, 0, s>>>(A.ws, A.N, npad, A.K, const_cast<uint8_t*>(A.sfb));
+  count_launches(2);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((A.N + BN - 1) / BN), (unsigned)((A.T + BM - 1) / BM), 1);
+  alignas(64) CUtensorMap ta, tb;
+  if (!make_codes_map(&ta, A.xq, A.T, A.K, BM) || !make_codes_map(&tb, A.wq, A.N, A.K, BN))
+    return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)(npad / BN), (unsigned)(tpad / BM), 1);
   timing_before(s);
-  w4a4_gemm_kernel<<<grid, GT, SMEM_BYTES, s>>>(A);
+  w4a4_gemm_kernel<<<grid, GT, SMEM_BYTES, s>>>(ta, tb, A);
   e = cudaGetLastError();
   timing_after(s);
   count_launches(1);

@@ -135,9 +135,11 @@ struct GemmArgs {
   float* y;               // [T, ldy] fp32
   int64_t T, N, K, ldy;
   unsigned* err_word;
+  const uint8_t* sfa;     // set by the launcher: interleaved scale factors (workspace)
+  const uint8_t* sfb;
 };
-size_t gemm_smem_bytes();
-cudaError_t launch_w4a4_gemm(const GemmArgs& A, cudaStream_t s);
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K);
+cudaError_t launch_w4a4_gemm(const GemmArgs& A, void* workspace, cudaStream_t s);
 
 cudaError_t launch_encode(const float* x, int64_t count, int codec, void* codes,
                           cudaStream_t s);

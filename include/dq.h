@@ -210,12 +210,17 @@ DQ_API dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int6
  *   w_scales        device [N, K/16] uint8 (its block_scales), 4-byte aligned
  *   w_tensor_scale  device [1] fp32 (its tensor_scale)
  *   y               device out [T, ldy] fp32, ldy >= N
- * Returns DQ_ERR_SHAPE if K is not a multiple of 64, DQ_ERR_UNSUPPORTED for another format;
- * a bounded wait that gives up raises DQ_ERR_TIMEOUT in the device error word. */
+ *   workspace       device scratch of dq_w4a4_gemm_workspace_bytes(T, N, K) bytes,
+ *                   16-byte aligned (the scale factors re-laid for the tensor core)
+ * Returns DQ_ERR_SHAPE if K is not a multiple of 64, DQ_ERR_UNSUPPORTED for another format,
+ * DQ_ERR_WORKSPACE for a missing or small workspace; a bounded wait that gives up raises
+ * DQ_ERR_TIMEOUT in the device error word. */
+DQ_API size_t dq_w4a4_gemm_workspace_bytes(int64_t T, int64_t N, int64_t K);
 DQ_API dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
                               const float* x_tensor_scale, int64_t T, const uint8_t* w_packed,
                               const uint8_t* w_scales, const float* w_tensor_scale, int64_t N,
-                              int64_t K, dq_format fmt, float* y, int64_t ldy, void* stream);
+                              int64_t K, dq_format fmt, float* y, int64_t ldy, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /* Codecs used by the kernels, exposed for bit-exact tests (one code per output element). */
 typedef enum {

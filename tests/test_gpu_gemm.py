@@ -99,6 +99,7 @@ def test_gemm_on_the_solver_and_activation_outputs(dq):
 def test_gemm_rejects_bad_shapes(dq):
     f = dq.fmt_of("NVFP4")
     nul = None
-    assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 96, f, nul, 8, nul) == 2
+    assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 96, f, nul, 8, nul, 0, nul) == 2
     assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 128, dq.fmt_of("MXFP4"), nul, 8,
-                           nul) == 8
+                           nul, 0, nul) == 8
+    assert dq.dq_w4a4_gemm_workspace_bytes(8, 8, 96) == 0
