@@ -108,6 +108,10 @@ def parse():
                     help="ablation: update both scales (the method), only r or only c")
     ap.add_argument("--qchange", action="store_true",
                     help="also record the per-iteration Q-change trace")
+    ap.add_argument("--gemm", action="store_true",
+                    help="time the W4A4 GEMM consumer instead: the 7 projections of block 0 "
+                         "(solved in NVFP4) against --gemm-tokens activation rows")
+    ap.add_argument("--gemm-tokens", type=int, default=8192)
     return ap.parse_args()
 
 
@@ -472,12 +476,112 @@ def run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elem
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
 
+def run_gemm(args, world, rank, local):
+    """W4A4 GEMM on the solver's and the activation quantizer's NVFP4 outputs: the 7
+    projections of the 8B layer set's block 0 against T activation rows each."""
+    import calibration_free_dual_b200 as dq
+    from calibration_free_dual_b200 import _lib
+    dev = torch.device("cuda", local)
+    cfg = wl.CONFIGS[CFG_ID]
+    layer = [e for e in cfg.layer_set() if e[0] == 0]
+    T = args.gemm_tokens
+    Ws = [wl.weight_device(cfg, b, p, device=dev, seed_offset=rank) for b, p, _, _ in layer]
+    sols = dq.solve_batched(Ws, "NVFP4", cfg.iters)
+    g = torch.Generator(device=dev)
+    g.manual_seed(77 + rank)
+    acts = []
+    for W, sol in zip(Ws, sols):
+        X = torch.randn((T, W.shape[1]), generator=g, device=dev).to(torch.bfloat16)
+        acts.append(dq.act_quant(X, "NVFP4", sol["c"]))
+    lib = _lib.get()
+    shapes = [(T, W.shape[0], W.shape[1]) for W in Ws]
+    need = max(lib.dq_w4a4_gemm_workspace_bytes(t, n, k) for t, n, k in shapes)
+    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    ys = [torch.empty((t, n), dtype=torch.float32, device=dev) for t, n, _ in shapes]
+    stream = torch.cuda.current_stream(dev)
+    sptr = ctypes.c_void_p(stream.cuda_stream)
+    f = dq.fmt_of("NVFP4")
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    def step():
+        for (t, n, k), a, sol, y in zip(shapes, acts, sols, ys):
+            st = lib.dq_w4a4_gemm(p(a["x_packed"]), p(a["scales"]), p(a["tensor_scale"]), t,
+                                  p(sol["q_packed"]), p(sol["block_scales"]),
+                                  p(sol["tensor_scale"]), n, k, f, p(y), n, p(ws), need, sptr)
+            if st != 0:
+                raise dq.DQError(st, "dq_w4a4_gemm")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    cap = 7 * args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+    for e in ev_s + ev_e:
+        e.record(stream)
+    arr_s = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_s])
+    arr_e = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_e])
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = lib.dq_kernel_launches()
+    lib.dq_set_timing_events(arr_s, arr_e, cap)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    used = lib.dq_timing_events_used()
+    lib.dq_set_timing_events(None, None, 0)
+    launches = lib.dq_kernel_launches() - launches0
+    barrier(world)
+    clk = clocks.stop()
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error during the timed region")
+    ms_total = reduce_max(t0.elapsed_time(t1), world)
+    kern_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s[:used], ev_e[:used]))
+    flop = 2.0 * sum(t * n * k for t, n, k in shapes)
+    ms_step = ms_total / args.steps
+    peaks, peak_src = _peaks()
+    fp4_peak = float(peaks["bf16_tflops"]) * 4.0          # dense FP4 / BF16 = 9 / 2.25
+    achieved = flop * args.steps / (kern_ms * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": "W4A4 GEMM TFLOP/s (NVFP4 operands from the solver and dq_act_quant)",
+            "value": world * flop / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": "block-0 projections of the Llama-3.1-8B-shaped layer set "
+                                   "(7 GEMMs, %d tokens each, K = 4096 / 14336)" % T,
+                       "step": "7 dq_w4a4_gemm calls (each: scale-factor re-layout + GEMM)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+                         "peak_source": "measured bf16 %.1f TF/s (%s) x 4, the nominal dense "
+                                        "FP4/BF16 ratio" % (float(peaks["bf16_tflops"]),
+                                                            peak_src),
+                         "kernel": "w4a4_gemm_kernel (the scale-factor re-layout launches "
+                                   "are outside this figure, inside ms_per_step)",
+                         "kernel_ms_per_step": kern_ms / args.steps},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.gemm:
+            run_gemm(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:
