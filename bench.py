@@ -283,9 +283,10 @@ def run_ours(args, world, rank, local):
     act_ws = torch.empty((256,), dtype=torch.uint8, device=dev)
     k0 = next(i for i, (b, p, _, _) in enumerate(layer) if b == 0 and p == 1)
 
-    def mats_for(Wlist):
-        arr = (_lib.dq_matrix * count)()
-        for i, (W, o) in enumerate(zip(Wlist, outs)):
+    def mats_for(Wlist, olist=None):
+        olist = outs if olist is None else olist
+        arr = (_lib.dq_matrix * len(Wlist))()
+        for i, (W, o) in enumerate(zip(Wlist, olist)):
             arr[i] = _lib.dq_matrix(W.data_ptr(), W.shape[0], W.shape[1], W.stride(0), None,
                                     None, o["q_packed"].data_ptr(), o["r"].data_ptr(),
                                     o["c"].data_ptr(), o["block_scales"].data_ptr(),
@@ -295,25 +296,33 @@ def run_ours(args, world, rank, local):
     mats = mats_for(Ws)
     sptr = ctypes.c_void_p(stream.cuda_stream)
 
-    def step(mats_arr, Xin):
+    def solve_call(mats_arr, n_mats, strm):
+        sp = ctypes.c_void_p(strm.cuda_stream)
         if opts is None:
-            st = lib.dq_solve_batched(mats_arr, count, _lib.DQ_BF16, fmt, T,
-                                      ctypes.c_void_p(ws.data_ptr()), ws_bytes, sptr)
+            st = lib.dq_solve_batched(mats_arr, n_mats, _lib.DQ_BF16, fmt, T,
+                                      ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
         else:
-            st = lib.dq_solve_batched_ex(mats_arr, count, _lib.DQ_BF16, fmt, T,
+            st = lib.dq_solve_batched_ex(mats_arr, n_mats, _lib.DQ_BF16, fmt, T,
                                          ctypes.byref(opts), ctypes.c_void_p(ws.data_ptr()),
-                                         ws_bytes, sptr)
+                                         ws_bytes, sp)
         if st != 0:
             raise dq.DQError(st, "dq_solve_batched")
+
+    def act_call(Xin, strm):
         st = lib.dq_act_quant(ctypes.c_void_p(Xin.data_ptr()), _lib.DQ_BF16, Xin.shape[0],
                               Xin.shape[1], Xin.stride(0),
                               ctypes.c_void_p(outs[k0]["c"].data_ptr()), fmt,
                               ctypes.c_void_p(act_out["x_packed"].data_ptr()),
                               ctypes.c_void_p(act_out["scales"].data_ptr()),
                               ctypes.c_void_p(act_out["tensor_scale"].data_ptr()),
-                              ctypes.c_void_p(act_ws.data_ptr()), act_ws.numel(), sptr)
+                              ctypes.c_void_p(act_ws.data_ptr()), act_ws.numel(),
+                              ctypes.c_void_p(strm.cuda_stream))
         if st != 0:
             raise dq.DQError(st, "dq_act_quant")
+
+    def step(mats_arr, Xin):
+        solve_call(mats_arr, count, stream)
+        act_call(Xin, stream)
 
     elems = sum(W.numel() for W in Ws)
     for _ in range(args.warmup):
@@ -386,7 +395,8 @@ def run_ours(args, world, rank, local):
     # ------------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elems, T)
+        e2e = run_e2e(args, world, dev, Ws, X, outs, act_out, solve_call, act_call, mats_for,
+                      layer, elems, T)
 
     # ------------------------------------------------------------------ CPU baseline
     cpu = None
@@ -431,8 +441,12 @@ def _group_sizes(layer):
     return [sizes[k] for k in order]
 
 
-def run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elems, T):
-    """Same step through the public API from pinned host buffers, results read back."""
+def run_e2e(args, world, dev, Ws, X, outs, act_out, solve_call, act_call, mats_for, layer,
+            elems, T):
+    """The same step through the public API from pinned host buffers, results read back to
+    pinned host buffers, pipelined the way a user streams a model: one dq_solve_batched per
+    block of the layer set on the compute stream, while a copy stream brings in the next
+    blocks' weights and another takes the finished blocks' outputs back."""
     host_W = [torch.empty(W.shape, dtype=W.dtype, pin_memory=True) for W in Ws]
     for h, W in zip(host_W, Ws):
         h.copy_(W)
@@ -440,7 +454,6 @@ def run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elem
     host_X.copy_(X)
     dev_W = [torch.empty_like(W) for W in Ws]
     dev_X = torch.empty_like(X)
-    mats = mats_for(dev_W)
     keys = ("q_packed", "block_scales", "c", "tensor_scale", "mse")
     host_out = [{k: torch.empty(o[k].shape, dtype=o[k].dtype, pin_memory=True) for k in keys}
                 for o in outs]
@@ -449,31 +462,60 @@ def run_e2e(args, world, dev, stream, Ws, X, outs, act_out, step, mats_for, elem
     h2d = sum(h.numel() * h.element_size() for h in host_W) + host_X.numel() * host_X.element_size()
     d2h = sum(o[k].numel() * o[k].element_size() for o in outs for k in keys) + \
         sum(v.numel() * v.element_size() for v in act_out.values())
+    blocks = sorted({b for b, _, _, _ in layer})
+    chunks = [[i for i, (b, _, _, _) in enumerate(layer) if b == blk] for blk in blocks]
+    chunk_mats = [mats_for([dev_W[i] for i in idx], [outs[i] for i in idx]) for idx in chunks]
+    comp = torch.cuda.current_stream(dev)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
 
     def e2e_step():
-        for h, d in zip(host_W, dev_W):
-            d.copy_(h, non_blocking=True)
-        dev_X.copy_(host_X, non_blocking=True)
-        step(mats, dev_X)
-        for o, ho in zip(outs, host_out):
-            for k in keys:
-                ho[k].copy_(o[k], non_blocking=True)
-        for k, v in act_out.items():
-            host_act[k].copy_(v, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(comp)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        ev_in = []
+        with torch.cuda.stream(s_in):
+            dev_X.copy_(host_X, non_blocking=True)
+            for idx in chunks:
+                for i in idx:
+                    dev_W[i].copy_(host_W[i], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_in)
+                ev_in.append(e)
+        for ci, idx in enumerate(chunks):
+            comp.wait_event(ev_in[ci])
+            solve_call(chunk_mats[ci], len(idx), comp)
+            if ci == 0:
+                act_call(dev_X, comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                for i in idx:
+                    for k in keys:
+                        host_out[i][k].copy_(outs[i][k], non_blocking=True)
+                if ci == 0:
+                    for k, v in act_out.items():
+                        host_act[k].copy_(v, non_blocking=True)
+        end = torch.cuda.Event()
+        end.record(s_out)
+        comp.wait_event(end)
 
     e2e_step()
     torch.cuda.synchronize(dev)
     barrier(world)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(comp)
     for _ in range(args.steps):
         e2e_step()
-    b.record(stream)
+    b.record(comp)
     torch.cuda.synchronize(dev)
     ms = reduce_max(a.elapsed_time(b), world) / args.steps
     return {"value": world * elems * T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "pipeline": "per block: H2D, dq_solve_batched and D2H on three streams"}
 
 
 def run_gemm(args, world, rank, local):
