@@ -19,7 +19,7 @@ LIB = os.path.join(PKG, "libdq.so")
 BUILD = os.path.join(ROOT, "_build")
 SOURCES = ["dq_api.cu", "dq_solve.cu", "dq_solve_ext.cu", "dq_solve_int8.cu",
            "dq_solve_int8_ext.cu", "dq_act.cu", "dq_codec.cu", "dq_noalloc.cu", "dq_gemm.cu"]
-HEADERS = ["dq_device.cuh", "dq_internal.h", "dq_solve_kernel.cuh"]
+HEADERS = ["dq_device.cuh", "dq_internal.h", "dq_solve_kernel.cuh", "dq_gemm.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -12,6 +12,7 @@
 
 #include "dq.h"
 #include "dq_internal.h"
+#include "dq_gemm.h"
 
 namespace {
 

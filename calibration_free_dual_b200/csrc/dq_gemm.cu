@@ -24,6 +24,7 @@
 
 #include "dq_device.cuh"
 #include "dq_internal.h"
+#include "dq_gemm.h"
 
 namespace dq {
 namespace {
