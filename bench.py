@@ -332,7 +332,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device error during warm-up")
 
     # per-launch events for the solve kernel over the timed region
-    per_step = sum((n + 31) // 32 for n in _group_sizes(layer))
+    per_step = sum((n + 63) // 64 for n in _group_sizes(layer))   # launches per step
     cap = per_step * args.steps
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
     ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]

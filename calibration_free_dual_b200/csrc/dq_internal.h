@@ -8,7 +8,7 @@
 namespace dq {
 
 constexpr int SOLVE_NT = 512;          // threads per CTA of the solve kernel (one CTA per SM)
-constexpr int SOLVE_MAXMATS = 32;      // matrices per solve launch (descriptors by value)
+constexpr int SOLVE_MAXMATS = 64;      // matrices per solve launch (descriptors by value)
 constexpr size_t SOLVE_SMEM_MAX = 227 * 1024;   // dynamic shared memory of one CTA
 
 struct SolveMat {
