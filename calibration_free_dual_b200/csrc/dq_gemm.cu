@@ -10,10 +10,13 @@
 //   * warp 0 (one lane) produces: per 256-wide K slice, two TMA tile loads (128-byte
 //     swizzle) of the packed E2M1 codes and bulk copies of the scale factors, all completing
 //     on the slice's "full" mbarrier; three slices in flight;
-//   * warp 1 (one lane) consumes: copies the slice's scale factors to TMEM (tcgen05.cp),
-//     issues the four MMAs and commits them to the slice's "empty" mbarrier;
-//   * warps 2-5 wait for the last commit, read the accumulator (tcgen05.ld), apply the two
-//     tensor scales and store fp32.
+//   * warps 2-5 move each slice's scale factors from shared memory into TMEM (tcgen05.st,
+//     one 32-lane sub-partition per warp) and signal the slice's "sf_ready" mbarrier, which
+//     keeps those copies out of the tensor pipe (tcgen05.cp there serialises with the MMAs);
+//   * warp 1 (one lane) issues the slice's four MMAs once both barriers have completed and
+//     commits them to the slice's "empty" mbarrier;
+//   * after the last commit, warps 2-5 read the accumulator (tcgen05.ld), apply the two
+//     tensor scales, stage the tile in the idle slice buffers and store it row by row.
 // The scale factors are first re-laid (a small pre-pass per operand) into the 128-row x 4
 // interleaving the tensor core reads, so a slice's scale factors are one contiguous copy.
 // Every mbarrier wait is bounded by the global timer; on timeout the kernel raises the error
@@ -29,35 +32,39 @@
 namespace dq {
 namespace {
 
-constexpr int GT = 192;                 // threads per CTA: producer, MMA, 4 epilogue warps
+constexpr int GT = 192;                 // threads per CTA: producer, MMA, 4 scale/epilogue warps
+constexpr unsigned FULL_MASK = 0xFFFFFFFFu;
 // 128 x 128 tiles with three K slices in flight let two CTAs share an SM, so one CTA's set-up
 // and epilogue overlap the other's MMAs: measured 10-20% faster than 128 x 256 tiles with
-// four slices and one CTA per SM (the code handles both tile widths)
+// four slices and one CTA per SM
 constexpr int BM = 128, BN = 128;       // output tile (tokens x weight rows)
-constexpr int NH = BN / 128;            // 128-row halves of the weight tile
-constexpr int BKE = 256;                // K elements per slice (4 MMAs of K = 64)
+constexpr int BKE = 256;                // K elements per slice (NKB MMAs of K = 64)
+constexpr int NKB = BKE / 64;
 constexpr int BKB = BKE / 2;            // bytes of packed E2M1 per row per slice (128)
 constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BKB;       // 16 KB
-constexpr int B_BYTES = BN * BKB;       // 32 KB
-constexpr int SFA_BYTES = BM * BKE / 16;   // 2 KB: 4 blocks of 512 (one per MMA)
-constexpr int SFB_BYTES = BN * BKE / 16;   // NH row halves x 4 blocks of 512
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 54 KB
+constexpr int B_BYTES = BN * BKB;       // 16 KB
+constexpr int SFA_BYTES = BM * BKE / 16;   // NKB blocks of 512 (one per MMA)
+constexpr int SFB_BYTES = BN * BKE / 16;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 36 KB
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
 constexpr int SMEM_NEED = BAR_OFF + 128 + 1024;    // barriers, TMEM slot, 1024-byte alignment
 // with two CTAs per SM, more than a third of the SM's shared memory keeps a third CTA (and its
 // TMEM allocation) off the SM
 constexpr int SMEM_BYTES = SMEM_NEED;
 constexpr uint32_t SF_COL0 = BN;                          // after the fp32 accumulator
-constexpr uint32_t SF_COLS_PER_STAGE = 16 + 16 * NH;      // SFA 4 x 4, SFB 4 x 4 NH
-constexpr uint32_t TMEM_COLS = (SF_COL0 + STAGES * SF_COLS_PER_STAGE) <= 256 ? 256 : 512;
-constexpr int CTAS_PER_SM = TMEM_COLS == 256 ? 2 : 1;
-constexpr int SMEM_LAUNCH = (CTAS_PER_SM == 2 && SMEM_BYTES < 80 * 1024) ? 80 * 1024 : SMEM_BYTES;
+constexpr uint32_t SF_COLS_PER_STAGE = 8 * NKB;           // SFA NKB MMAs x 4, SFB NKB x 4
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int CTAS_PER_SM = 2;
+constexpr int SMEM_LAUNCH = SMEM_BYTES < 80 * 1024 ? 80 * 1024 : SMEM_BYTES;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;   // 2 s: far beyond any slice's work
 
+static_assert(NKB == 2 || NKB == 4, "slice of 2 or 4 MMAs");
 static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned slices (128-byte swizzle)");
 static_assert(SMEM_LAUNCH * CTAS_PER_SM <= 226 * 1024, "shared memory");
 static_assert(SF_COL0 + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns");
+static_assert(8 * (3 * STAGES + 1) + 8 <= 128, "barrier block");
+static_assert(BM * BN * 4 <= STAGES * STAGE_BYTES, "epilogue staging fits in the slice buffers");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -139,13 +146,34 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 // K-major operand slice written by a 128-byte-swizzled TMA box of 128-byte rows: 8-row
 // groups 1024 bytes apart; an MMA's K = 64 slice starts 32 bytes further per step
 __device__ __forceinline__ uint64_t operand_desc(uint32_t addr) { return smem_desc(addr, 16, 1024, 2); }
-// scale factors: 32 rows x 16 bytes, 8-row groups 128 bytes apart, no swizzle
-__device__ __forceinline__ uint64_t sf_desc(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
-// 32 rows x 128 bits of scale factors from shared memory to TMEM, replicated into the four
-// 32-lane sub-partitions
-__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(sdesc)
-               : "memory");
+// 32 lanes x N consecutive 32-bit columns (N = 16 or 32) from registers into this warp's
+// TMEM sub-partition
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 32) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+           "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+           "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+           "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+           "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+  } else {
+    static_assert(N == 16, "16 or 32 columns");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16};"
+        :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+           "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+           "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+  }
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 // D (+)= A x B^T with E2M1 operands and E4M3 scale factors per 16 elements
 __device__ __forceinline__ void mma_nvfp4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -181,25 +209,43 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 
-// instruction descriptor: A, B E2M1 (1), scale factors UE4M3 (0), K-major, M = 128, N = 256
+// instruction descriptor: A, B E2M1 (1), scale factors UE4M3 (0), K-major, M = BM, N = BN
 constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(BM >> 4) << 24);
 
 // Scale codes [rows, K/16] -> [row block of 128][K/64][512 bytes]: in each 512-byte block the
 // four scales of row r of the block (for one MMA's 64 elements) sit at (r % 32) * 16 +
-// (r / 32) * 4, the layout tcgen05.cp 32x128b.warpx4 expects. Rows in [rows, rows_pad) are 0.
-__global__ void sf_interleave_kernel(const uint8_t* __restrict__ src, int64_t rows,
-                                     int64_t rows_pad, int64_t K, uint8_t* __restrict__ dst) {
+// (r / 32) * 4, so lane l of every TMEM sub-partition takes the 16 bytes at l * 16 and the
+// tensor core picks the 4 bytes of its row group. Rows in [rows, rows_pad) are 0.
+// One CTA re-lays SF_G groups of 4 scale bytes for one block of 128 rows of one operand
+// (blockIdx.x: activation row blocks first, then weight row blocks; blockIdx.y: group chunk)
+// through shared memory, with row-contiguous reads and block-contiguous writes.
+constexpr int SF_G = 32;
+__global__ void __launch_bounds__(256)
+sf_interleave_kernel(const uint8_t* __restrict__ xs, int64_t T, int64_t tblk,
+                     const uint8_t* __restrict__ ws, int64_t N, int64_t K,
+                     uint8_t* __restrict__ sfa, uint8_t* __restrict__ sfb) {
+  __shared__ uint32_t tile[SF_G][129];                 // [group][output word], padded
   const int64_t kq = K / 64;
-  const int64_t total = rows_pad * kq;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = i / kq, g = i % kq;
+  const bool act = (int64_t)blockIdx.x < tblk;
+  const int64_t rb = act ? (int64_t)blockIdx.x : (int64_t)blockIdx.x - tblk;
+  const uint8_t* src = act ? xs : ws;
+  const int64_t rows = act ? T : N;
+  uint8_t* dst = act ? sfa : sfb;
+  const int64_t g0 = (int64_t)blockIdx.y * SF_G;
+  const int ng = (int)((kq - g0) < SF_G ? (kq - g0) : SF_G);
+  for (int i = threadIdx.x; i < 128 * SF_G; i += blockDim.x) {
+    const int r = i / SF_G, gg = i % SF_G;
+    const int64_t row = rb * 128 + r;
     uint32_t v = 0u;
-    if (row < rows) v = *reinterpret_cast<const uint32_t*>(src + row * (K / 16) + 4 * g);
-    const int r = (int)(row & 127);
-    uint8_t* blk = dst + ((row >> 7) * kq + g) * 512;
-    *reinterpret_cast<uint32_t*>(blk + (r & 31) * 16 + (r >> 5) * 4) = v;
+    if (gg < ng && row < rows)
+      v = *reinterpret_cast<const uint32_t*>(src + row * (K / 16) + 4 * (g0 + gg));
+    tile[gg][(r & 31) * 4 + (r >> 5)] = v;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < ng * 128; i += blockDim.x) {
+    const int gg = i / 128, w = i % 128;
+    reinterpret_cast<uint32_t*>(dst + (rb * kq + g0 + gg) * 512)[w] = tile[gg][w];
   }
 }
 
@@ -212,17 +258,19 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;               // 1024-byte aligned slices
   unsigned char* base_ptr = smem_raw + (sbase - raw);
-  const uint32_t full0 = sbase + BAR_OFF;                      // full[s]  = full0 + 8s
-  const uint32_t empty0 = full0 + 8 * STAGES;                  // empty[s] = empty0 + 8s
-  const uint32_t accbar = empty0 + 8 * STAGES;                 // accumulator complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BAR_OFF + 8 * (2 * STAGES + 1));
-  volatile int* fail = reinterpret_cast<volatile int*>(base_ptr + BAR_OFF + 8 * (2 * STAGES + 2));
+  const uint32_t full0 = sbase + BAR_OFF;                      // full[s]    = full0 + 8s
+  const uint32_t empty0 = full0 + 8 * STAGES;                  // empty[s]   = empty0 + 8s
+  const uint32_t sfrdy0 = empty0 + 8 * STAGES;                 // sf_ready[s] = sfrdy0 + 8s
+  const uint32_t accbar = sfrdy0 + 8 * STAGES;                 // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BAR_OFF + 8 * (3 * STAGES + 1));
+  volatile int* fail = reinterpret_cast<volatile int*>(base_ptr + BAR_OFF + 8 * (3 * STAGES + 2));
 
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
   if (tid == 32) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
+      mbar_init(sfrdy0 + 8 * s, 4);
     }
     mbar_init(accbar, 1);
     *fail = 0;
@@ -242,70 +290,110 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const uint32_t use = (uint32_t)(k / STAGES);             // how often slot s was used
       if (!mbar_wait(empty0 + 8 * s, (use & 1u) ^ 1u)) { *fail = 1; break; }
       if (*fail) break;
-      const int nkb = (int)((kq - 4ll * k) < 4 ? (kq - 4ll * k) : 4);
+      const int nkb = (int)((kq - (int64_t)NKB * k) < NKB ? (kq - (int64_t)NKB * k) : NKB);
       const uint32_t sf_bytes = 512u * nkb;
       const uint32_t st = sbase + s * STAGE_BYTES;
-      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES + (1 + NH) * sf_bytes);
+      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES + 2 * sf_bytes);
       tma_load_2d(st, &tmA, k * BKB, (int)t0, full0 + 8 * s);
       tma_load_2d(st + A_BYTES, &tmB, k * BKB, (int)n0, full0 + 8 * s);
-      bulk_load(st + A_BYTES + B_BYTES, A.sfa + ((t0 >> 7) * kq + 4ll * k) * 512, sf_bytes,
+      bulk_load(st + A_BYTES + B_BYTES, A.sfa + ((t0 >> 7) * kq + (int64_t)NKB * k) * 512, sf_bytes,
                 full0 + 8 * s);
-      for (int h = 0; h < NH; ++h)
-        bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + 2048 * h,
-                  A.sfb + (((n0 >> 7) + h) * kq + 4ll * k) * 512, sf_bytes, full0 + 8 * s);
+      bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, A.sfb + ((n0 >> 7) * kq + (int64_t)NKB * k) * 512,
+                sf_bytes, full0 + 8 * s);
     }
   } else if (warp == 1 && lane == 0) {
-    // ---- MMA issue
+    // ---- MMA issue: the slice's operands (full) and its scale factors in TMEM (sf_ready)
     bool ok = true;
     for (int k = 0; k < nk; ++k) {
       const int s = k % STAGES;
-      const uint32_t use = (uint32_t)(k / STAGES);
-      if (!mbar_wait(full0 + 8 * s, use & 1u) || *fail) { *fail = 1; ok = false; break; }
-      tc_fence_after();
-      const int nkb = (int)((kq - 4ll * k) < 4 ? (kq - 4ll * k) : 4);
-      const uint32_t st = sbase + s * STAGE_BYTES;
-      // SFA of MMA kb: 4 columns at +4kb; SFB: 4 NH columns at +16 + 4 NH kb (half h at +4h)
-      const uint32_t tsf = tmem + SF_COL0 + SF_COLS_PER_STAGE * s;
-      for (int kb = 0; kb < nkb; ++kb) {
-        tmem_cp_sf(tsf + 4 * kb, sf_desc(st + A_BYTES + B_BYTES + kb * 512));
-        for (int h = 0; h < NH; ++h)
-          tmem_cp_sf(tsf + 16 + 4 * NH * kb + 4 * h,
-                     sf_desc(st + A_BYTES + B_BYTES + SFA_BYTES + 2048 * h + kb * 512));
+      const uint32_t par = (uint32_t)(k / STAGES) & 1u;
+      if (!mbar_wait(full0 + 8 * s, par) || !mbar_wait(sfrdy0 + 8 * s, par) || *fail) {
+        *fail = 1;
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      const int nkb = (int)((kq - (int64_t)NKB * k) < NKB ? (kq - (int64_t)NKB * k) : NKB);
+      const uint32_t st = sbase + s * STAGE_BYTES;
+      // SFA of MMA kb: TMEM columns +4kb; SFB: +4NKB +4kb
+      const uint32_t tsf = tmem + SF_COL0 + SF_COLS_PER_STAGE * s;
       for (int kb = 0; kb < nkb; ++kb)
         mma_nvfp4(tmem, operand_desc(st + 32 * kb), operand_desc(st + A_BYTES + 32 * kb),
                   IDESC_NVFP4, (k > 0 || kb > 0) ? 1u : 0u, tsf + 4 * kb,
-                  tsf + 16 + 4 * NH * kb);
+                  tsf + 4 * NKB + 4 * kb);
       mma_commit(empty0 + 8 * s);
     }
     if (ok) mma_commit(accbar);
   } else if (warp >= 2) {
-    // ---- epilogue: TMEM sub-partition warp % 4 holds rows 32 * (warp % 4) ...
+    // TMEM sub-partition warp % 4: lanes (and accumulator rows) 32 * (warp % 4) ...
     const int sp = warp & 3;
-    bool ok = false;
-    if (lane == 0) ok = mbar_wait(accbar, 0) && !*fail;
-    ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+    const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
+    // ---- scale factors of every slice into TMEM. Each 512-byte block holds the scales of
+    // one MMA for 128 rows, row r at (r % 32) * 16 + (r / 32) * 4: every sub-partition gets
+    // the same 16 bytes per lane, and the tensor core picks the 4 bytes of its row group.
+    bool ok = true;
+    for (int k = 0; k < nk && ok; ++k) {
+      const int s = k % STAGES;
+      const uint32_t par = (uint32_t)(k / STAGES) & 1u;
+      int got = 0;
+      if (lane == 0) got = (mbar_wait(full0 + 8 * s, par) && !*fail) ? 1 : 0;
+      ok = __shfl_sync(FULL_MASK, got, 0) != 0;
+      if (!ok) break;
+      const unsigned char* sfs = base_ptr + s * STAGE_BYTES + A_BYTES + B_BYTES + lane * 16;
+      uint32_t r[8 * NKB];
+#pragma unroll
+      for (int kb = 0; kb < NKB; ++kb) {
+        const uint4 a = *reinterpret_cast<const uint4*>(sfs + kb * 512);
+        const uint4 b = *reinterpret_cast<const uint4*>(sfs + SFA_BYTES + kb * 512);
+        r[4 * kb + 0] = a.x; r[4 * kb + 1] = a.y; r[4 * kb + 2] = a.z; r[4 * kb + 3] = a.w;
+        r[4 * NKB + 4 * kb + 0] = b.x; r[4 * NKB + 4 * kb + 1] = b.y;
+        r[4 * NKB + 4 * kb + 2] = b.z; r[4 * NKB + 4 * kb + 3] = b.w;
+      }
+      tmem_st<8 * NKB>(lane_base + SF_COL0 + SF_COLS_PER_STAGE * s, r);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfrdy0 + 8 * s);
+    }
+    // ---- epilogue: accumulator -> scaled fp32 -> this warp's 32 rows of a staging tile in
+    // the (now idle) slice buffers -> row-contiguous stores of the output tile
+    if (ok) {
+      int got = 0;
+      if (lane == 0) got = (mbar_wait(accbar, 0) && !*fail) ? 1 : 0;
+      ok = __shfl_sync(FULL_MASK, got, 0) != 0;
+    }
     if (ok) {
       tc_fence_after();
       const float scale = __fmul_rn(*A.xst, *A.wst);
-      const int64_t t = t0 + sp * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)(sp * 32) << 16);
+      // 32 rows x BN fp32, 16-byte chunks XOR-swizzled by row so that both the row-per-lane
+      // writes and the row-per-warp reads are free of bank conflicts
+      float4* stage = reinterpret_cast<float4*>(base_ptr) + sp * 32 * (BN / 4);
 #pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
         float v[32];
-        tmem_ld32(lane_addr + cb * 32, v);
-        if (t < A.T) {
-          float* yrow = A.y + t * A.ldy + n0 + cb * 32;
-          const int64_t rem = A.N - n0 - cb * 32;
-          const int64_t ncols = rem < 32 ? rem : 32;
-          if (ncols == 32 && (reinterpret_cast<uintptr_t>(yrow) & 15u) == 0) {
+        tmem_ld32(lane_base + cb * 32, v);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(yrow + i) =
-                  make_float4(v[i] * scale, v[i + 1] * scale, v[i + 2] * scale, v[i + 3] * scale);
-          } else {
-            for (int i = 0; i < ncols; ++i) yrow[i] = v[i] * scale;
-          }
+        for (int j = 0; j < 8; ++j)
+          stage[lane * (BN / 4) + ((cb * 8 + j) ^ (lane & 7))] =
+              make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale,
+                          v[4 * j + 3] * scale);
+      }
+      __syncwarp();
+      const int64_t c0 = n0 + 4 * lane;                          // this lane's 4 columns
+      const int64_t ncols = A.N - c0;                            // columns left from c0
+      const bool vec = ((A.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(A.y) & 15u) == 0);
+#pragma unroll 4
+      for (int rr = 0; rr < 32; ++rr) {
+        const int64_t t = t0 + sp * 32 + rr;
+        if (t >= A.T) break;
+        const float4 o = stage[rr * (BN / 4) + (lane ^ (rr & 7))];
+        float* dst = A.y + t * A.ldy + c0;
+        if (ncols >= 4 && vec) {
+          *reinterpret_cast<float4*>(dst) = o;
+        } else {
+          if (ncols > 0) dst[0] = o.x;
+          if (ncols > 1) dst[1] = o.y;
+          if (ncols > 2) dst[2] = o.z;
+          if (ncols > 3) dst[3] = o.w;
         }
       }
     } else if (lane == 0) {
@@ -371,13 +459,12 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& A0, void* workspace, cudaStream_t s
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   A.sfa = ws;
   A.sfb = ws + tpad * (A.K / 16);
-  // re-lay both operands' scale factors
-  const int64_t work_a = tpad * (A.K / 64), work_b = npad * (A.K / 64);
-  const int ga = (int)std::min<int64_t>((work_a + 255) / 256, 148 * 8);
-  const int gb = (int)std::min<int64_t>((work_b + 255) / 256, 148 * 8);
-  sf_interleave_kernel<<<ga, 256, 0, s>>>(A.xs, A.T, tpad, A.K, const_cast<uint8_t*>(A.sfa));
-  sf_interleave_kernel<<<gb, 256, 0, s>>>(A.ws, A.N, npad, A.K, const_cast<uint8_t*>(A.sfb));
-  count_launches(2);
+  // re-lay both operands' scale factors (one launch)
+  const dim3 sfgrid((unsigned)(tpad / BM + npad / BN), (unsigned)((A.K / 64 + SF_G - 1) / SF_G), 1);
+  sf_interleave_kernel<<<sfgrid, 256, 0, s>>>(A.xs, A.T, tpad / BM, A.ws, A.N, A.K,
+                                              const_cast<uint8_t*>(A.sfa),
+                                              const_cast<uint8_t*>(A.sfb));
+  count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   alignas(64) CUtensorMap ta, tb;

@@ -55,7 +55,10 @@ def _check(y, xc, xs, sx, wc, ws, sw, K):
 
 
 @pytest.mark.parametrize("T,N,K", [(128, 128, 256), (256, 384, 1024), (200, 136, 320),
-                                   (1, 8, 64), (130, 260, 4096)])
+                                   (1, 8, 64), (130, 260, 4096),
+                                   # 40 groups of 64 (a ragged 32-group re-layout chunk), an
+                                   # output row pitch that is not a multiple of 4 floats
+                                   (67, 130, 2560)])
 def test_gemm_matches_oracle(dq, T, N, K):
     rng = np.random.default_rng(T * 7 + N + K)
     xc, xs = _operand(rng, T, K, zero_frac=0.05)
