@@ -7,14 +7,14 @@
 // sm_100a design: 5th-generation tensor cores, block-scaled, warp-specialized. One CTA (six
 // warps, two per SM) owns a 128 x 128 output tile accumulated in tensor memory (TMEM) by
 // tcgen05.mma.kind::mxf4nvf4.block_scale (M = 128, N = 128, K = 64 per instruction):
-//   * warp 0 (one lane) produces: per 256-wide K slice, two TMA tile loads (128-byte
-//     swizzle) of the packed E2M1 codes and bulk copies of the scale factors, all completing
-//     on the slice's "full" mbarrier; three slices in flight;
+//   * warp 0 (one lane) produces: per 256-wide K slice, bulk copies of the scale factors
+//     (completing on the slice's "sf_full" mbarrier) and two TMA tile loads (128-byte
+//     swizzle) of the packed E2M1 codes (on its "full" mbarrier); three slices in flight;
 //   * warps 2-5 move each slice's scale factors from shared memory into TMEM (tcgen05.st,
 //     one 32-lane sub-partition per warp) and signal the slice's "sf_ready" mbarrier, which
 //     keeps those copies out of the tensor pipe (tcgen05.cp there serialises with the MMAs);
-//   * warp 1 (one lane) issues the slice's four MMAs once both barriers have completed and
-//     commits them to the slice's "empty" mbarrier;
+//   * warp 1 (one lane) issues the slice's four MMAs once "full" and "sf_ready" have
+//     completed and commits them to the slice's "empty" mbarrier;
 //   * after the last commit, warps 2-5 read the accumulator (tcgen05.ld), apply the two
 //     tensor scales, stage the tile in the idle slice buffers and store it row by row.
 // The scale factors are first re-laid (a small pre-pass per operand) into the 128-row x 4
@@ -23,6 +23,7 @@
 // word, frees its TMEM and returns.
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
 #include <cuda.h>   // CUtensorMap and its enums (the encoder is fetched from the driver)
 
 #include "dq_device.cuh"
@@ -63,7 +64,7 @@ static_assert(NKB == 2 || NKB == 4, "slice of 2 or 4 MMAs");
 static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned slices (128-byte swizzle)");
 static_assert(SMEM_LAUNCH * CTAS_PER_SM <= 226 * 1024, "shared memory");
 static_assert(SF_COL0 + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "TMEM columns");
-static_assert(8 * (3 * STAGES + 1) + 8 <= 128, "barrier block");
+static_assert(8 * (4 * STAGES + 1) + 8 <= 128, "barrier block");
 static_assert(BM * BN * 4 <= STAGES * STAGE_BYTES, "epilogue staging fits in the slice buffers");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -83,6 +84,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// shared -> global tile store through a tensor map (bulk-group completion)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+      :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(src) : "memory");
 }
 
 // ---- mbarrier
@@ -251,7 +259,7 @@ sf_interleave_kernel(const uint8_t* __restrict__ xs, int64_t T, int64_t tblk,
 
 __global__ void __launch_bounds__(GT, CTAS_PER_SM)
 w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ GemmArgs A) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ GemmArgs A) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t t0 = (int64_t)blockIdx.y * BM, n0 = (int64_t)blockIdx.x * BN;
@@ -261,9 +269,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const uint32_t full0 = sbase + BAR_OFF;                      // full[s]    = full0 + 8s
   const uint32_t empty0 = full0 + 8 * STAGES;                  // empty[s]   = empty0 + 8s
   const uint32_t sfrdy0 = empty0 + 8 * STAGES;                 // sf_ready[s] = sfrdy0 + 8s
-  const uint32_t accbar = sfrdy0 + 8 * STAGES;                 // accumulator complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BAR_OFF + 8 * (3 * STAGES + 1));
-  volatile int* fail = reinterpret_cast<volatile int*>(base_ptr + BAR_OFF + 8 * (3 * STAGES + 2));
+  const uint32_t sffull0 = sfrdy0 + 8 * STAGES;                // sf_full[s]  = sffull0 + 8s
+  const uint32_t accbar = sffull0 + 8 * STAGES;                // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + BAR_OFF + 8 * (4 * STAGES + 1));
+  volatile int* fail = reinterpret_cast<volatile int*>(base_ptr + BAR_OFF + 8 * (4 * STAGES + 2));
 
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
   if (tid == 32) {
@@ -271,6 +280,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
       mbar_init(sfrdy0 + 8 * s, 4);
+      mbar_init(sffull0 + 8 * s, 1);
     }
     mbar_init(accbar, 1);
     *fail = 0;
@@ -293,13 +303,16 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int nkb = (int)((kq - (int64_t)NKB * k) < NKB ? (kq - (int64_t)NKB * k) : NKB);
       const uint32_t sf_bytes = 512u * nkb;
       const uint32_t st = sbase + s * STAGE_BYTES;
-      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES + 2 * sf_bytes);
+      // the small scale-factor copies first, on their own barrier: their trip into TMEM
+      // overlaps the operand tiles' arrival
+      mbar_expect_tx(sffull0 + 8 * s, 2 * sf_bytes);
+      bulk_load(st + A_BYTES + B_BYTES, A.sfa + ((t0 >> 7) * kq + (int64_t)NKB * k) * 512, sf_bytes,
+                sffull0 + 8 * s);
+      bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, A.sfb + ((n0 >> 7) * kq + (int64_t)NKB * k) * 512,
+                sf_bytes, sffull0 + 8 * s);
+      mbar_expect_tx(full0 + 8 * s, A_BYTES + B_BYTES);
       tma_load_2d(st, &tmA, k * BKB, (int)t0, full0 + 8 * s);
       tma_load_2d(st + A_BYTES, &tmB, k * BKB, (int)n0, full0 + 8 * s);
-      bulk_load(st + A_BYTES + B_BYTES, A.sfa + ((t0 >> 7) * kq + (int64_t)NKB * k) * 512, sf_bytes,
-                full0 + 8 * s);
-      bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES, A.sfb + ((n0 >> 7) * kq + (int64_t)NKB * k) * 512,
-                sf_bytes, full0 + 8 * s);
     }
   } else if (warp == 1 && lane == 0) {
     // ---- MMA issue: the slice's operands (full) and its scale factors in TMEM (sf_ready)
@@ -336,7 +349,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       const int s = k % STAGES;
       const uint32_t par = (uint32_t)(k / STAGES) & 1u;
       int got = 0;
-      if (lane == 0) got = (mbar_wait(full0 + 8 * s, par) && !*fail) ? 1 : 0;
+      if (lane == 0) got = (mbar_wait(sffull0 + 8 * s, par) && !*fail) ? 1 : 0;
       ok = __shfl_sync(FULL_MASK, got, 0) != 0;
       if (!ok) break;
       const unsigned char* sfs = base_ptr + s * STAGE_BYTES + A_BYTES + B_BYTES + lane * 16;
@@ -354,8 +367,11 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(sfrdy0 + 8 * s);
     }
-    // ---- epilogue: accumulator -> scaled fp32 -> this warp's 32 rows of a staging tile in
-    // the (now idle) slice buffers -> row-contiguous stores of the output tile
+    // ---- epilogue: accumulator -> scaled fp32 -> this warp's 32 rows, staged in the (now
+    // idle) slice buffers as four 32 x 32 blocks of 128-byte rows, 16-byte chunks XOR-swizzled
+    // by row (the 128-byte TMA swizzle: conflict-free writes of a row per lane) -> TMA tensor
+    // stores of the four blocks (rows and columns past T, N clipped), or, when the output's
+    // pitch or base does not allow a tensor map, row-contiguous stores by the warp
     if (ok) {
       int got = 0;
       if (lane == 0) got = (mbar_wait(accbar, 0) && !*fail) ? 1 : 0;
@@ -364,36 +380,51 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (ok) {
       tc_fence_after();
       const float scale = __fmul_rn(*A.xst, *A.wst);
-      // 32 rows x BN fp32, 16-byte chunks XOR-swizzled by row so that both the row-per-lane
-      // writes and the row-per-warp reads are free of bank conflicts
-      float4* stage = reinterpret_cast<float4*>(base_ptr) + sp * 32 * (BN / 4);
+      unsigned char* stage = base_ptr + sp * (BN / 32) * 4096;   // 1024-byte aligned blocks
 #pragma unroll 1
       for (int cb = 0; cb < BN / 32; ++cb) {
         float v[32];
         tmem_ld32(lane_base + cb * 32, v);
+        float4* blk = reinterpret_cast<float4*>(stage + cb * 4096);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          stage[lane * (BN / 4) + ((cb * 8 + j) ^ (lane & 7))] =
+          blk[lane * 8 + (j ^ (lane & 7))] =
               make_float4(v[4 * j] * scale, v[4 * j + 1] * scale, v[4 * j + 2] * scale,
                           v[4 * j + 3] * scale);
       }
-      __syncwarp();
-      const int64_t c0 = n0 + 4 * lane;                          // this lane's 4 columns
-      const int64_t ncols = A.N - c0;                            // columns left from c0
-      const bool vec = ((A.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(A.y) & 15u) == 0);
+      if (A.store_tma) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          for (int cb = 0; cb < BN / 32; ++cb)
+            if (n0 + cb * 32 < A.N && t0 + sp * 32 < A.T)        // boxes wholly outside: none
+              tma_store_2d(&tmY, smem_u32(stage + cb * 4096), (int)(n0 + cb * 32),
+                           (int)(t0 + sp * 32));
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        }
+        __syncwarp();
+      } else {
+        __syncwarp();
+        const int cb = lane >> 3, j = lane & 7;                   // this lane's 4 columns
+        const int64_t c0 = n0 + cb * 32 + 4 * j;
+        const int64_t ncols = A.N - c0;                           // columns left from c0
+        const bool vec = ((A.ldy & 3) == 0) && ((reinterpret_cast<uintptr_t>(A.y) & 15u) == 0);
+        const float4* blk = reinterpret_cast<const float4*>(stage + cb * 4096);
 #pragma unroll 4
-      for (int rr = 0; rr < 32; ++rr) {
-        const int64_t t = t0 + sp * 32 + rr;
-        if (t >= A.T) break;
-        const float4 o = stage[rr * (BN / 4) + (lane ^ (rr & 7))];
-        float* dst = A.y + t * A.ldy + c0;
-        if (ncols >= 4 && vec) {
-          *reinterpret_cast<float4*>(dst) = o;
-        } else {
-          if (ncols > 0) dst[0] = o.x;
-          if (ncols > 1) dst[1] = o.y;
-          if (ncols > 2) dst[2] = o.z;
-          if (ncols > 3) dst[3] = o.w;
+        for (int rr = 0; rr < 32; ++rr) {
+          const int64_t t = t0 + sp * 32 + rr;
+          if (t >= A.T) break;
+          const float4 o = blk[rr * 8 + (j ^ (rr & 7))];
+          float* dst = A.y + t * A.ldy + c0;
+          if (ncols >= 4 && vec) {
+            *reinterpret_cast<float4*>(dst) = o;
+          } else {
+            if (ncols > 0) dst[0] = o.x;
+            if (ncols > 1) dst[1] = o.y;
+            if (ncols > 2) dst[2] = o.z;
+            if (ncols > 3) dst[3] = o.w;
+          }
         }
       }
     } else if (lane == 0) {
@@ -444,6 +475,20 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
          CUDA_SUCCESS;
 }
 
+// y [rows, ldy] fp32, box of 32 rows x 32 floats (128 bytes), 128-byte swizzle; needs a
+// 16-byte aligned base and a row pitch of a multiple of 16 bytes
+bool make_out_map(CUtensorMap* map, float* y, int64_t rows, int64_t cols, int64_t ldy) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(y) & 15u) != 0 || (ldy & 3) != 0) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ldy * 4)};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
@@ -467,15 +512,17 @@ cudaError_t launch_w4a4_gemm(const GemmArgs& A0, void* workspace, cudaStream_t s
   count_launches(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  alignas(64) CUtensorMap ta, tb;
+  alignas(64) CUtensorMap ta, tb, ty;
   if (!make_codes_map(&ta, A.xq, A.T, A.K, BM) || !make_codes_map(&tb, A.wq, A.N, A.K, BN))
     return cudaErrorInvalidValue;
+  A.store_tma = make_out_map(&ty, A.y, A.T, A.N, A.ldy) ? 1 : 0;
+  if (!A.store_tma) memset(&ty, 0, sizeof(ty));          // not read by the kernel
   e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SMEM_LAUNCH);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)(npad / BN), (unsigned)(tpad / BM), 1);
   timing_before(s);
-  w4a4_gemm_kernel<<<grid, GT, SMEM_LAUNCH, s>>>(ta, tb, A);
+  w4a4_gemm_kernel<<<grid, GT, SMEM_LAUNCH, s>>>(ta, tb, ty, A);
   e = cudaGetLastError();
   timing_after(s);
   count_launches(1);

@@ -20,6 +20,7 @@ struct GemmArgs {
   unsigned* err_word;
   const uint8_t* sfa;     // set by the launcher: interleaved scale factors (workspace)
   const uint8_t* sfb;
+  int store_tma;          // set by the launcher: y is written by TMA tensor stores
 };
 size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K);
 cudaError_t launch_w4a4_gemm(const GemmArgs& A, void* workspace, cudaStream_t s);
