@@ -36,9 +36,6 @@ constexpr float NVFP4_TENSOR_DIV = 2688.0f;   // 6 (E2M1 max) * 448 (E4M3 max)
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t u) {
   return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
-__device__ __forceinline__ bool bf16x2_nonfinite(uint32_t u) {
-  return ((u & 0x7F80u) == 0x7F80u) || ((u & 0x7F800000u) == 0x7F800000u);
-}
 
 // ------------------------------------------------------------------ E2M1 elements
 // Two binary32 values -> one byte of two E2M1 codes (low nibble = lo), RNE, saturating.

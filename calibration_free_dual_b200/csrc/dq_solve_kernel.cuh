@@ -195,6 +195,25 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     else reinterpret_cast<uint8_t*>(pcodes_v)[code0 + k * (NT / LPB)] = (uint8_t)code;
   };
 
+  // ---- rows [0, R) into shared memory (their only read from HBM) by asynchronous 16-byte
+  // copies, all in flight at once; rows past m (only in the last sweep) are zero-filled and
+  // add nothing to any sum. Issued first, awaited before the first pass; the iteration-0
+  // pass checks every row for non-finite values.
+  {
+    constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
+    const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
+    const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(Wsm));
+#pragma unroll 4
+    for (int ch = tid; ch < L.R * CH; ch += NT) {
+      const int row = ch / CH, part = ch % CH;
+      const bool in = row < m;
+      const char* src = base + (int64_t)(in ? row : 0) * pitch + part * 16;
+      const uint32_t dst = dst0 + 16u * chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                   :: "r"(dst), "l"(src), "r"(in ? 16 : 0) : "memory");
+    }
+  }
+
   // ---- tensor scale (NVFP4) and the code -> (r, 1/r) table
   float s_t = 1.0f;
   if constexpr (SCALE == SCALE_E4M3) {
@@ -221,29 +240,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     icvec[tid] = __frcp_rn(cj);
   }
 
-  // ---- rows [0, R) into shared memory (their only read from HBM); rows past m (only in the
-  // last sweep) are zeros, which add nothing to any sum
-  {
-    constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
-    const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
-    uint4* dst = reinterpret_cast<uint4*>(Wsm);
-    bool bad = false;
-#pragma unroll 4
-    for (int ch = tid; ch < L.R * CH; ch += NT) {
-      const int row = ch / CH, part = ch % CH;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row < m) v = ldg_stream(base + (int64_t)row * pitch + part * 16);
-      if constexpr (ESZ == 2) {
-        bad |= bf16x2_nonfinite(v.x) | bf16x2_nonfinite(v.y) | bf16x2_nonfinite(v.z) |
-               bf16x2_nonfinite(v.w);
-      } else {
-        bad |= ((v.x & 0x7F800000u) == 0x7F800000u) | ((v.y & 0x7F800000u) == 0x7F800000u) |
-               ((v.z & 0x7F800000u) == 0x7F800000u) | ((v.w & 0x7F800000u) == 0x7F800000u);
-      }
-      dst[chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ)] = v;
-    }
-    if (bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
-  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
   float2 cc[8], ic[8];
@@ -346,14 +343,17 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       float2 w[8];
       unpack<ESZ>(buf, w);
       ScaleVal sc;
-      if constexpr (!INIT) sc = scn;
-      const uint32_t old_code = sc.code;
+      uint32_t old_code = 0u;                 // the Q-change trace's previous scale code
+      if constexpr (!INIT) {
+        sc = scn;
+        old_code = sc.code;
+      }
       if (k + 1 < RPT) {
         fetch(k + 1, buf);
         if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
       }
       if constexpr (INIT) {
-        if (k >= KS) bad |= nonfinite8(w);
+        bad |= nonfinite8(w);
         float a = 0.0f;
 #pragma unroll
         for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
