@@ -16,9 +16,11 @@
 //   * warp 1 (one lane) issues the slice's four MMAs once "full" and "sf_ready" have
 //     completed and commits them to the slice's "empty" mbarrier;
 //   * after the last commit, warps 2-5 read the accumulator (tcgen05.ld), apply the two
-//     tensor scales, stage the tile in the idle slice buffers and store it row by row.
-// The scale factors are first re-laid (a small pre-pass per operand) into the 128-row x 4
-// interleaving the tensor core reads, so a slice's scale factors are one contiguous copy.
+//     tensor scales, stage the tile in the idle slice buffers as 32 x 32 blocks and write
+//     them with TMA tensor stores (row stores when the output allows no tensor map).
+// The scale factors are first re-laid (one small pre-pass launch for both operands) into the
+// 128-row x 4 interleaving the tensor core reads, so a slice's scale factors are one
+// contiguous copy.
 // Every mbarrier wait is bounded by the global timer; on timeout the kernel raises the error
 // word, frees its TMEM and returns.
 #include <algorithm>
