@@ -531,9 +531,10 @@ def run_gemm(args, world, rank, local):
     sols = dq.solve_batched(Ws, "NVFP4", cfg.iters)
     g = torch.Generator(device=dev)
     g.manual_seed(77 + rank)
-    acts = []
+    acts, Xs = [], []
     for W, sol in zip(Ws, sols):
         X = torch.randn((T, W.shape[1]), generator=g, device=dev).to(torch.bfloat16)
+        Xs.append(X)
         acts.append(dq.act_quant(X, "NVFP4", sol["c"]))
     lib = _lib.get()
     shapes = [(T, W.shape[0], W.shape[1]) for W in Ws]
@@ -588,6 +589,34 @@ def run_gemm(args, world, rank, local):
     ms_total = reduce_max(t0.elapsed_time(t1), world)
     kern_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s[:used], ev_e[:used]))
     flop = 2.0 * sum(t * n * k for t, n, k in shapes)
+
+    # the same layers from the unquantized activations: dq_w4a4_linear (fl32(X * c) quantized
+    # straight into the tensor core's layouts, the weight's scale factors re-laid, the GEMM)
+    need_lin = max(lib.dq_w4a4_linear_workspace_bytes(t, n, k, f) for t, n, k in shapes)
+    wsl = torch.empty((need_lin,), dtype=torch.uint8, device=dev)
+
+    def lin_step():
+        for (t, n, k), X, sol, y in zip(shapes, Xs, sols, ys):
+            st = lib.dq_w4a4_linear(p(X), 1, t, k, k, p(sol["c"]), p(sol["q_packed"]),
+                                    p(sol["block_scales"]), p(sol["tensor_scale"]), n, f, p(y),
+                                    n, p(wsl), need_lin, sptr)
+            if st != 0:
+                raise dq.DQError(st, "dq_w4a4_linear")
+
+    for _ in range(args.warmup):
+        lin_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    l0 = torch.cuda.Event(enable_timing=True)
+    l1 = torch.cuda.Event(enable_timing=True)
+    l0.record(stream)
+    for _ in range(args.steps):
+        lin_step()
+    l1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error during the timed linear region")
+    lin_ms = reduce_max(l0.elapsed_time(l1), world) / args.steps
     ms_step = ms_total / args.steps
     peaks, peak_src = _peaks()
     fp4_peak = float(peaks["bf16_tflops"]) * 4.0          # dense FP4 / BF16 = 9 / 2.25
@@ -610,6 +639,11 @@ def run_gemm(args, world, rank, local):
                          "kernel": "w4a4_gemm_kernel (the scale-factor re-layout launches "
                                    "are outside this figure, inside ms_per_step)",
                          "kernel_ms_per_step": kern_ms / args.steps},
+            "linear": {"ms_per_step": lin_ms,
+                       "value": world * flop / (lin_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "step": "7 dq_w4a4_linear calls from bf16 X and c (activation "
+                               "quantized into the tensor core's layouts, weight scale "
+                               "factors re-laid, GEMM); timed after the GEMM region"},
             "gpu_launches": int(launches),
             "clocks": clk,
         }

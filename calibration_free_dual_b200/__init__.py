@@ -16,7 +16,8 @@ from ._lib import (DQ_OK, DQ_INT4, DQ_MXINT4, DQ_MXFP4, DQ_NVFP4, DQ_INT8,  # no
                    DQ_UPDATE_BOTH, DQ_UPDATE_ROW_ONLY, DQ_UPDATE_COL_ONLY,
                    dq_format, dq_matrix, dq_solve_options)
 from .api import (DQError, FORMATS, fmt_of, solve, solve_batched, act_quant, encode,  # noqa: F401
-                  decode, last_device_error, w4a4_gemm)
+                  decode, last_device_error, w4a4_gemm,
+                  w4a4_linear)
 
 
 def __getattr__(name):

@@ -61,6 +61,10 @@ SIGNATURES = {
     "dq_w4a4_gemm": (c_int32, [c_void_p, c_void_p, c_void_p, c_int64, c_void_p, c_void_p,
                                c_void_p, c_int64, c_int64, dq_format, c_void_p, c_int64,
                                c_void_p, c_size_t, c_void_p]),
+    "dq_w4a4_linear_workspace_bytes": (c_size_t, [c_int64, c_int64, c_int64, dq_format]),
+    "dq_w4a4_linear": (c_int32, [c_void_p, c_int32, c_int64, c_int64, c_int64, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_int64, dq_format, c_void_p,
+                                 c_int64, c_void_p, c_size_t, c_void_p]),
     "dq_encode": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p]),
     "dq_decode": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p]),
     "dq_last_device_error": (c_int32, [c_void_p]),

@@ -236,6 +236,38 @@ def w4a4_gemm(x: dict, w: dict, fmt="NVFP4", stream=None,
     return y
 
 
+def w4a4_linear(X: torch.Tensor, w: dict, c: torch.Tensor | None = None, fmt="NVFP4",
+                stream=None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """dq_w4a4_linear: y[T, N] = quantized fl32(X * c) times a solve's output `w`
+    (q_packed, block_scales, tensor_scale), the activation quantized in the GEMM's layouts."""
+    _need_cuda(X, "X")
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be 2-D row-major")
+    f = fmt_of(fmt)
+    wq, ws, wst = w["q_packed"], w["block_scales"], w["tensor_scale"]
+    for t, name in ((wq, "q_packed"), (ws, "block_scales")):
+        _need_cuda(t, name)
+        if not t.is_contiguous():
+            raise ValueError(name + " must be contiguous")
+    T, K = X.shape
+    N = wq.shape[0]
+    if wq.shape[1] * 2 != K:
+        raise ValueError("activation and weight K differ")
+    if c is not None:
+        _need_cuda(c, "c")
+    y = torch.empty((T, N), dtype=torch.float32, device=X.device)
+    lib = _lib.get()
+    need = lib.dq_w4a4_linear_workspace_bytes(T, N, K, f)
+    if need == 0:
+        raise DQError(_lib.DQ_ERR_SHAPE, "NVFP4 and K a multiple of 64 required")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=X.device)
+    _check(lib.dq_w4a4_linear(_p(X), _dtype_code(X), T, K, X.stride(0), _p(c), _p(wq), _p(ws),
+                              _p(wst), N, f, _p(y), N, _p(workspace), need,
+                              _stream_ptr(stream)), "dq_w4a4_linear")
+    return y
+
+
 _CODE_DTYPE = {_lib.DQ_CODEC_BF16: torch.int16}
 
 

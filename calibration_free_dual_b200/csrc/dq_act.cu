@@ -138,8 +138,20 @@ __global__ void act_quant_kernel(const ActLaunch A) {
         else
           *reinterpret_cast<uint32_t*>(A.x_packed + row * qpitch + col / 2) = (uint32_t)packed;
         if ((lane % LB) == 0) {
-          if constexpr (SCB == 2) reinterpret_cast<uint16_t*>(A.scales)[row * nb + col / B] = (uint16_t)code;
-          else reinterpret_cast<uint8_t*>(A.scales)[row * nb + col / B] = (uint8_t)code;
+          const int64_t b = col / B;
+          if constexpr (SCB == 2) {
+            reinterpret_cast<uint16_t*>(A.scales)[row * nb + b] = (uint16_t)code;
+          } else if constexpr (SCALE == SCALE_E4M3) {
+            // the W4A4 GEMM's layout: [row / 128][n / 64][512 bytes], the four scales of a
+            // 64-channel group of row r at (r % 32) * 16 + (r % 128 / 32) * 4
+            const int64_t r = row & 127;
+            const int64_t off = A.sf_tc ? ((row >> 7) * (A.n / 64) + (b >> 2)) * 512 +
+                                              (r & 31) * 16 + (r >> 5) * 4 + (b & 3)
+                                        : row * nb + b;
+            reinterpret_cast<uint8_t*>(A.scales)[off] = (uint8_t)code;
+          } else {
+            reinterpret_cast<uint8_t*>(A.scales)[row * nb + b] = (uint8_t)code;
+          }
         }
       }
     }

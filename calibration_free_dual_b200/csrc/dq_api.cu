@@ -335,7 +335,7 @@ dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
   if (!aligned16(workspace)) return DQ_ERR_INVALID_ARG;
   unsigned* errp = nullptr;
   if ((st = err_word_ptr(&errp)) != DQ_OK) return st;
-  dq::GemmArgs A;
+  dq::GemmArgs A = {};
   A.xq = x_packed;
   A.xs = x_scales;
   A.xst = x_tensor_scale;
@@ -379,7 +379,7 @@ dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, 
   unsigned* errp = nullptr;
   if ((st = err_word_ptr(&errp)) != DQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dq::ActLaunch A;
+  dq::ActLaunch A = {};
   A.X = X;
   A.tokens = tokens;
   A.n = n;
@@ -394,6 +394,94 @@ dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, 
     if ((st = from_cuda(cudaMemsetAsync(workspace, 0, 4, s))) != DQ_OK) return st;
   }
   return from_cuda(dq::launch_act(A, fmt.kind, fmt.group, esize, s));
+}
+
+// W4A4 linear layer: workspace = [amax word, activation tensor scale | activation codes |
+// activation scale factors in the tensor core's layout | weight scale factors re-laid]
+namespace {
+struct LinearWs {
+  size_t codes, sfa, sfb, total;
+};
+LinearWs linear_ws(int64_t T, int64_t N, int64_t K) {
+  LinearWs l;
+  const int64_t tpad = (T + 127) / 128 * 128;
+  l.codes = 256;
+  l.sfa = dq::align_up(l.codes + (size_t)T * (size_t)(K / 2), 256);
+  l.sfb = dq::align_up(l.sfa + (size_t)tpad * (size_t)(K / 16), 256);
+  l.total = l.sfb + dq::gemm_workspace_bytes(T, N, K, true);
+  return l;
+}
+}  // namespace
+
+size_t dq_w4a4_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, dq_format fmt) {
+  if (check_format(fmt) != DQ_OK || fmt.kind != DQ_NVFP4) return 0;
+  if (T <= 0 || N <= 0 || K <= 0 || K % 64 != 0) return 0;
+  return linear_ws(T, N, K).total;
+}
+
+dq_status dq_w4a4_linear(const void* X, int32_t dtype, int64_t T, int64_t K, int64_t ldx,
+                         const float* c, const uint8_t* w_packed, const uint8_t* w_scales,
+                         const float* w_tensor_scale, int64_t N, dq_format fmt, float* y,
+                         int64_t ldy, void* workspace, size_t workspace_bytes, void* stream) {
+  dq_status st = check_format(fmt);
+  if (st != DQ_OK) return st;
+  if (fmt.kind != DQ_NVFP4) return DQ_ERR_UNSUPPORTED;
+  const int esize = dtype_size(dtype);
+  if (esize == 0) return DQ_ERR_DTYPE;
+  if (T <= 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return DQ_ERR_INVALID_ARG;
+  if (K % 64 != 0) return DQ_ERR_SHAPE;
+  if (T > ((int64_t)1 << 30) || N > ((int64_t)1 << 30) || K > ((int64_t)1 << 30))
+    return DQ_ERR_SHAPE;
+  if (X == nullptr || w_packed == nullptr || w_scales == nullptr || w_tensor_scale == nullptr ||
+      y == nullptr)
+    return DQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || (ldx * esize) % 16 != 0) return DQ_ERR_INVALID_ARG;
+  if (c != nullptr && !aligned16(c)) return DQ_ERR_INVALID_ARG;
+  if (!aligned16(w_packed) || (reinterpret_cast<uintptr_t>(w_scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(y) & 3u))
+    return DQ_ERR_INVALID_ARG;
+  const LinearWs l = linear_ws(T, N, K);
+  if (workspace == nullptr || workspace_bytes < l.total) return DQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DQ_ERR_INVALID_ARG;
+  unsigned* errp = nullptr;
+  if ((st = err_word_ptr(&errp)) != DQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t kq = K / 64;
+  // the amax word, and the scale factors of the rows past T in the last 128-row block
+  if ((st = from_cuda(cudaMemsetAsync(ws, 0, 4, s))) != DQ_OK) return st;
+  if (T % 128 != 0 &&
+      (st = from_cuda(cudaMemsetAsync(ws + l.sfa + (T / 128) * kq * 512, 0, (size_t)kq * 512, s))) != DQ_OK)
+    return st;
+  // one pass over X: fl32(X * c) quantized, codes and scale factors in the GEMM's layouts
+  dq::ActLaunch act = {};
+  act.X = X;
+  act.tokens = T;
+  act.n = K;
+  act.ldx = ldx;
+  act.c = c;
+  act.x_packed = ws + l.codes;
+  act.scales = ws + l.sfa;
+  act.tensor_scale = reinterpret_cast<float*>(ws + 4);
+  act.amax_bits = reinterpret_cast<unsigned*>(ws);
+  act.err_word = errp;
+  act.sf_tc = 1;
+  if ((st = from_cuda(dq::launch_act(act, fmt.kind, fmt.group, esize, s))) != DQ_OK) return st;
+  dq::GemmArgs A = {};
+  A.xq = ws + l.codes;
+  A.xs = nullptr;
+  A.xst = reinterpret_cast<const float*>(ws + 4);
+  A.wq = w_packed;
+  A.ws = w_scales;
+  A.wst = w_tensor_scale;
+  A.y = y;
+  A.T = T;
+  A.N = N;
+  A.K = K;
+  A.ldy = ldy;
+  A.err_word = errp;
+  A.sfa = ws + l.sfa;
+  return from_cuda(dq::launch_w4a4_gemm(A, ws + l.sfb, s));
 }
 
 dq_status dq_encode(const float* x, int64_t count, int32_t codec, void* codes, void* stream) {

@@ -495,20 +495,22 @@ int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
-size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K) {
-  // interleaved scale factors: activation rows padded to 128, weight rows to 256
-  return (size_t)(round_up(T, BM) + round_up(N, BN)) * (size_t)(K / 16) + 256;
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, bool sfa_given) {
+  // interleaved scale factors, rows padded to whole 128-row blocks
+  return (size_t)((sfa_given ? 0 : round_up(T, BM)) + round_up(N, BN)) * (size_t)(K / 16) + 256;
 }
 
 cudaError_t launch_w4a4_gemm(const GemmArgs& A0, void* workspace, cudaStream_t s) {
   GemmArgs A = A0;
   const int64_t tpad = round_up(A.T, BM), npad = round_up(A.N, BN);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  A.sfa = ws;
-  A.sfb = ws + tpad * (A.K / 16);
-  // re-lay both operands' scale factors (one launch)
-  const dim3 sfgrid((unsigned)(tpad / BM + npad / BN), (unsigned)((A.K / 64 + SF_G - 1) / SF_G), 1);
-  sf_interleave_kernel<<<sfgrid, 256, 0, s>>>(A.xs, A.T, tpad / BM, A.ws, A.N, A.K,
+  const bool sfa_given = A.sfa != nullptr;
+  if (!sfa_given) A.sfa = ws;
+  A.sfb = sfa_given ? ws : ws + tpad * (A.K / 16);
+  // re-lay the scale factors (one launch; the weight's only when the activation's are given)
+  const int64_t tblk = sfa_given ? 0 : tpad / BM;
+  const dim3 sfgrid((unsigned)(tblk + npad / BN), (unsigned)((A.K / 64 + SF_G - 1) / SF_G), 1);
+  sf_interleave_kernel<<<sfgrid, 256, 0, s>>>(A.xs, A.T, tblk, A.ws, A.N, A.K,
                                               const_cast<uint8_t*>(A.sfa),
                                               const_cast<uint8_t*>(A.sfb));
   count_launches(1);

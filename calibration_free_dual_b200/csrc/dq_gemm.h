@@ -18,11 +18,15 @@ struct GemmArgs {
   float* y;               // [T, ldy] fp32
   int64_t T, N, K, ldy;
   unsigned* err_word;
-  const uint8_t* sfa;     // set by the launcher: interleaved scale factors (workspace)
+  // interleaved scale factors [rows / 128][K / 64][512 bytes]: sfb is set by the launcher
+  // (workspace); sfa too when null on entry, else the activation's are already laid out there
+  // (rows past T zero) and xs is not read
+  const uint8_t* sfa;
   const uint8_t* sfb;
   int store_tma;          // set by the launcher: y is written by TMA tensor stores
 };
-size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K);
+// sfa_given: the activation's scale factors come laid out (workspace for the weight's only)
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, bool sfa_given = false);
 cudaError_t launch_w4a4_gemm(const GemmArgs& A, void* workspace, cudaStream_t s);
 
 }  // namespace dq

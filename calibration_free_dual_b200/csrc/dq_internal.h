@@ -121,6 +121,7 @@ struct ActLaunch {
   float* tensor_scale;
   unsigned* amax_bits;
   unsigned* err_word;
+  int sf_tc;          // NVFP4: scales in the tensor core's layout (see dq_gemm.h), else [tokens, n/16]
 };
 cudaError_t launch_act(const ActLaunch& A, int kind, int group, int esize, cudaStream_t s);
 

@@ -222,6 +222,29 @@ DQ_API dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
                               int64_t K, dq_format fmt, float* y, int64_t ldy, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* W4A4 linear layer from the unquantized activation: the activation rescale + quantization
+ * (dq_act_quant, NVFP4) as the producer of the W4A4 GEMM (dq_w4a4_gemm) in one call. One
+ * pass over X forms x~ = fl32(X * c), quantizes it per (token, 16 channels) and writes the
+ * codes and scale factors straight in the layouts the tensor core reads (no re-layout of the
+ * activation's scale factors); the GEMM then consumes them with the solver's weight codes.
+ * The result is bit-identical to dq_act_quant followed by dq_w4a4_gemm.
+ *   X               device [T, ldx] (dtype), 16-byte aligned, ldx*esize % 16 == 0, ldx >= K
+ *   c               device [K] fp32 (the solver's c) or NULL, 16-byte aligned
+ *   w_packed, w_scales, w_tensor_scale, N, fmt, y, ldy: as for dq_w4a4_gemm (K = in
+ *                   features, a multiple of 64)
+ *   workspace       device scratch of dq_w4a4_linear_workspace_bytes(T, N, K, fmt) bytes,
+ *                   16-byte aligned (the quantized activation and both operands' scale
+ *                   factors in the tensor core's layout)
+ * Errors as for dq_act_quant and dq_w4a4_gemm; a non-finite x~ raises DQ_ERR_NONFINITE in
+ * the device error word. dq_w4a4_linear_workspace_bytes returns 0 for an unsupported format
+ * or shape. */
+DQ_API size_t dq_w4a4_linear_workspace_bytes(int64_t T, int64_t N, int64_t K, dq_format fmt);
+DQ_API dq_status dq_w4a4_linear(const void* X, int32_t dtype, int64_t T, int64_t K,
+                                int64_t ldx, const float* c, const uint8_t* w_packed,
+                                const uint8_t* w_scales, const float* w_tensor_scale, int64_t N,
+                                dq_format fmt, float* y, int64_t ldy, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Codecs used by the kernels, exposed for bit-exact tests (one code per output element). */
 typedef enum {
   DQ_CODEC_INT4 = 0,   /* RNE to -7..7, saturating; code = two's-complement nibble (uint8) */

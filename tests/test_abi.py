@@ -125,3 +125,27 @@ def test_solve_options_validation_and_workspace(dq):
     null_trace = dq._lib.dq_solve_options(dq.DQ_UPDATE_BOTH, (ctypes.c_void_p * 1)(None))
     assert dq.dq_solve_batched_ex(mats, 1, dq.DQ_BF16, f, 16, ctypes.byref(null_trace), None,
                                   0, None) == 1
+
+
+def test_linear_validation_and_workspace(dq):
+    """dq_w4a4_linear: format, shape, pointer and workspace checks before any CUDA call; the
+    workspace holds the quantized activation and both operands' scale factors."""
+    nv, mx = dq.fmt_of("NVFP4"), dq.fmt_of("MXFP4")
+    nul = None
+    assert dq.dq_w4a4_linear_workspace_bytes(130, 260, 96, nv) == 0          # K % 64
+    assert dq.dq_w4a4_linear_workspace_bytes(130, 260, 4096, mx) == 0        # NVFP4 only
+    need = dq.dq_w4a4_linear_workspace_bytes(130, 260, 4096, nv)
+    # codes 130 x 2048, activation scale factors 2 blocks of 128 rows, weight's 3 blocks
+    assert need >= 130 * 2048 + (256 + 384) * 256
+    assert dq.dq_w4a4_linear(nul, 1, 8, 96, 96, nul, nul, nul, nul, 8, nv, nul, 8, nul, 0,
+                             nul) == 2
+    assert dq.dq_w4a4_linear(nul, 1, 8, 128, 128, nul, nul, nul, nul, 8, mx, nul, 8, nul, 0,
+                             nul) == 8
+    assert dq.dq_w4a4_linear(nul, 1, 8, 128, 128, nul, nul, nul, nul, 8, nv, nul, 8, nul, 0,
+                             nul) == 1
+    assert dq.dq_w4a4_linear(nul, 9, 8, 128, 128, nul, nul, nul, nul, 8, nv, nul, 8, nul, 0,
+                             nul) == 3
+    assert dq.dq_w4a4_linear(0x1000, 1, 8, 128, 64, nul, 0x1000, 0x1000, 0x1000, 8, nv,
+                             0x1000, 8, nul, 0, nul) == 1                      # ldx < K
+    assert dq.dq_w4a4_linear(0x1000, 1, 8, 128, 128, nul, 0x1000, 0x1000, 0x1000, 8, nv,
+                             0x1000, 8, nul, 0, nul) == 4                      # no workspace

@@ -106,3 +106,53 @@ def test_gemm_rejects_bad_shapes(dq):
     assert dq.dq_w4a4_gemm(nul, nul, nul, 8, nul, nul, nul, 8, 128, dq.fmt_of("MXFP4"), nul, 8,
                            nul, 0, nul) == 8
     assert dq.dq_w4a4_gemm_workspace_bytes(8, 8, 96) == 0
+
+
+def _weight(dq, rng, N, K):
+    """A solved NVFP4 weight (codes, block scales, tensor scale as dq_solve returns them)."""
+    w = rng.standard_t(4, (N, K)) * 0.014
+    W = torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16).cuda()
+    return dq.solve(W, "NVFP4", 4)
+
+
+@pytest.mark.parametrize("T,N,K,ldx_pad,with_c", [(130, 260, 4096, 0, True), (1, 8, 64, 0, True),
+                                                  (256, 384, 1024, 64, True),
+                                                  (67, 130, 2560, 0, False),
+                                                  (200, 136, 320, 32, True)])
+def test_linear_is_act_quant_then_gemm_bit_for_bit(dq, T, N, K, ldx_pad, with_c):
+    """dq_w4a4_linear (one quantization pass writing the tensor core's layouts, then the GEMM)
+    equals dq_act_quant followed by dq_w4a4_gemm exactly: ragged token blocks (their padded
+    scale rows zero), a strided X, no c, an output pitch that is not a multiple of 4 floats."""
+    rng = np.random.default_rng(T + 3 * N + K)
+    sol = _weight(dq, rng, N, K)
+    X = rng.standard_normal((T, K + ldx_pad)).astype(np.float32)
+    X[:, rng.choice(K, min(6, K), replace=False)] *= 50.0
+    Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()[:, :K]
+    c = sol["c"] if with_c else None
+    y1 = dq.w4a4_linear(Xd, sol, c)
+    act = dq.act_quant(Xd, "NVFP4", c)
+    y2 = dq.w4a4_gemm(act, sol)
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    assert torch.equal(y1, y2)
+
+
+def test_linear_matches_the_oracle_composition(dq):
+    """Against the oracle: its activation quantizer on fl32(X * c), then its GEMM of the two
+    sets of codes, within the GEMM's binary32 accumulation bound."""
+    rng = np.random.default_rng(21)
+    T, N, K = 150, 256, 1024
+    sol = _weight(dq, rng, N, K)
+    X = rng.standard_normal((T, K)).astype(np.float32)
+    X[:, rng.choice(K, 6, replace=False)] *= 50.0
+    Xt = torch.from_numpy(X).to(torch.bfloat16)
+    y = dq.w4a4_linear(Xt.cuda(), sol, sol["c"])
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    y = y.cpu().numpy().astype(np.float64)
+    from oracle import actquant as AQ
+    a = AQ.act_quant(Xt.float().numpy(), NV, sol["c"].cpu().numpy())
+    wc = F.unpack_codes(sol["q_packed"].cpu().numpy())
+    ws = sol["block_scales"].cpu().numpy()
+    sw = sol["tensor_scale"].cpu().numpy()[0]
+    _check(y, a["codes"], a["scale_codes"], a["s_t"], wc, ws, sw, K)
