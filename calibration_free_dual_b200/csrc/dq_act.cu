@@ -46,6 +46,14 @@ __device__ __forceinline__ void load8(const void* X, int64_t row, int64_t ldx, i
   }
 }
 
+// max that propagates NaN (a NaN operand gives NaN): the running |x| maximum of a block is
+// non-finite exactly when one of its elements is, so one test per block suffices
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 __device__ __forceinline__ void rescale8(const float* c, int64_t col, float (&x)[8]) {
   if (c == nullptr) return;
   const float4 a = __ldg(reinterpret_cast<const float4*>(c + col));
@@ -61,22 +69,29 @@ __global__ void act_amax_kernel(const ActLaunch A) {
   const int64_t warp0 = (int64_t)blockIdx.x * ACT_WARPS + threadIdx.x / 32;
   const int64_t nwarps = (int64_t)gridDim.x * ACT_WARPS;
   float a = 0.0f;
-  bool bad = false;
   for (int64_t row = warp0; row < A.tokens; row += nwarps) {
     for (int64_t col = 8 * lane; col < A.n; col += 256) {
       float x[8];
       load8<F32IN>(A.X, row, A.ldx, col, x);
       rescale8(A.c, col, x);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        bad |= !isfinite(x[k]);
-        a = fmaxf(a, fabsf(x[k]));
-      }
+      for (int k = 0; k < 8; ++k) a = max_nan(a, fabsf(x[k]));
     }
   }
+  const bool bad = !isfinite(a);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
-  if (lane == 0 && a > 0.0f) atomicMax(A.amax_bits, __float_as_uint(a));
+  // one atomic per CTA: the maxima of its warps meet in shared memory first (every warp of
+  // the launch updating one word serialises at its L2 slice)
+  __shared__ float wmax[ACT_WARPS];
+  if (lane == 0) wmax[threadIdx.x / 32] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < ACT_WARPS; ++w) m = fmaxf(m, wmax[w]);
+    if (m > 0.0f) atomicMax(A.amax_bits, __float_as_uint(m));
+  }
   if (bad) atomicOr(A.err_word, ERRBIT_NONFINITE);
 }
 
@@ -110,10 +125,8 @@ __global__ void act_quant_kernel(const ActLaunch A) {
       }
       float a = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        bad |= !isfinite(x[k]);
-        a = fmaxf(a, fabsf(x[k]));
-      }
+      for (int k = 0; k < 8; ++k) a = max_nan(a, fabsf(x[k]));
+      bad |= !isfinite(a);
 #pragma unroll
       for (int off = 1; off < LB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
       uint32_t code = 0;

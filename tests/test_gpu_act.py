@@ -93,8 +93,14 @@ def test_act_quant_config_sqnr(dq):
         assert all(np.isfinite(v) and v > 5 for v in res.values()), res
 
 
-def test_act_nonfinite_reported(dq):
-    X = torch.randn(8, 64)
-    X[2, 3] = float("inf")
-    dq.act_quant(X.cuda(), "MXFP4")
-    assert dq.last_device_error() == 5
+@pytest.mark.parametrize("fmt_name", ["MXFP4", "NVFP4", "INT4"])
+@pytest.mark.parametrize("bad", [float("inf"), float("-inf"), float("nan")])
+def test_act_nonfinite_reported(dq, fmt_name, bad):
+    """A non-finite channel anywhere in a block (first, middle, last element) is reported,
+    also through the NVFP4 amax pass and through the linear path."""
+    for col in (0, 37, 127):
+        X = torch.randn(8, 128)
+        X[2, col] = bad
+        dq.act_quant(X.cuda(), fmt_name)
+        assert dq.last_device_error() == 5
+    assert dq.last_device_error() == 0
