@@ -15,6 +15,7 @@ from __future__ import annotations
 import argparse
 import ctypes
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -112,6 +113,10 @@ def parse():
                     help="time the W4A4 GEMM consumer instead: the 7 projections of block 0 "
                          "(solved in NVFP4) against --gemm-tokens activation rows")
     ap.add_argument("--gemm-tokens", type=int, default=8192)
+    ap.add_argument("--act", action="store_true",
+                    help="time the activation rescale + quantization alone instead: 8192 x "
+                         "4096 bf16 activations with a k_proj's c, NVFP4 and INT4 g=128, L2 "
+                         "flushed before every call; SQNR with and without c")
     return ap.parse_args()
 
 
@@ -650,6 +655,101 @@ def run_gemm(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+ACT_BYTES_PER_ELEM = {"NVFP4": 2.0 + 0.5 + 1.0 / 16, "INT4": 2.0 + 0.5 + 2.0 / 128}
+
+
+def _act_decode(dq, out, fmt, T, n):
+    """Decoded activation d * q (binary32) from dq_act_quant's outputs, with the library's
+    own codecs on the device."""
+    from calibration_free_dual_b200 import _lib
+    xp = out["x_packed"]
+    nib = torch.stack((xp & 0xF, xp >> 4), dim=2).reshape(T, n).contiguous()
+    if fmt == "NVFP4":
+        q = dq.decode(nib, _lib.DQ_CODEC_E2M1)
+        d = dq.decode(out["scales"], _lib.DQ_CODEC_E4M3) * out["tensor_scale"][0]
+        B = 16
+    else:
+        q = dq.decode(nib, _lib.DQ_CODEC_INT4)
+        d = dq.decode(out["scales"], _lib.DQ_CODEC_BF16)
+        B = 128
+    return d.repeat_interleave(B, dim=1) * q
+
+
+def _sqnr(xt, xhat):
+    xt = xt.double()
+    err = ((xt - xhat.double()) ** 2).sum().item()
+    sig = (xt * xt).sum().item()
+    return float("inf") if err == 0.0 else 10.0 * math.log10(sig / err)
+
+
+def run_act(args, world, rank, local):
+    """dq_act_quant alone on the activation workload: 8192 tokens x 4096 bf16 channels
+    (N(0,1), six channels x50) rescaled by the c of a 1024 x 4096 k_proj (Student-t(4),
+    std 0.02, 1% columns x8, MXFP4, 16 iterations), quantized to NVFP4 and INT4 g=128."""
+    import calibration_free_dual_b200 as dq
+    from calibration_free_dual_b200 import _lib
+    dev = torch.device("cuda", local)
+    Wk = wl.weight_device(wl.ACT_KPROJ, 0, 1, device=dev, seed_offset=rank)
+    c = dq.solve(Wk, "MXFP4", wl.ACT_KPROJ.iters)["c"]
+    X = wl.act_device(seed=wl.ACT_SEED + rank, device=dev)
+    T, n = X.shape
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)    # 2x the 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    lib = _lib.get()
+    peaks, peak_src = _peaks()
+    res = {}
+    launches = 0
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    for fmt in ("NVFP4", "INT4"):
+        for _ in range(args.warmup):
+            dq.act_quant(X, fmt, c)
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world)
+        l0 = lib.dq_kernel_launches()
+        for e0, e1 in evs:
+            flush.fill_(1)                     # L2 holds none of X when the call starts
+            e0.record(stream)
+            out = dq.act_quant(X, fmt, c)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        launches += lib.dq_kernel_launches() - l0
+        if dq.last_device_error() != 0:
+            raise RuntimeError("device error during the timed region")
+        ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
+        sq = {"with_c": _sqnr(X.float() * c, _act_decode(dq, out, fmt, T, n))}
+        out0 = dq.act_quant(X, fmt, None)
+        sq["without_c"] = _sqnr(X.float(), _act_decode(dq, out0, fmt, T, n))
+        gbs = ACT_BYTES_PER_ELEM[fmt] * T * n / (ms * 1e-3) / 1e9
+        res[fmt] = {"ms_per_call": ms, "elems_per_s": world * T * n / (ms * 1e-3),
+                    "sqnr_db": sq,
+                    "roofline": {"bound": "hbm", "achieved": gbs,
+                                 "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                 "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
+                                 "bytes_per_elem": ACT_BYTES_PER_ELEM[fmt],
+                                 "peak_source": peak_src}}
+    clk = clocks.stop()
+    if rank == 0:
+        head = res["NVFP4"]
+        line = {
+            "metric": "activation rescale+quantize elements/s",
+            "value": head["elems_per_s"], "unit": "elem/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_call"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) "
+                                   "times a k_proj's c (1024 x 4096, MXFP4 solve), NVFP4 "
+                                   "(amax pass + quantization pass); INT4 g=128 alongside",
+                       "l2": "flushed (256 MB written) before every timed call"},
+            "roofline": dict(head["roofline"], kernel="act_amax_kernel + act_quant_kernel"),
+            "formats": res, "gpu_launches": int(launches), "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
@@ -658,6 +758,8 @@ def main():
             run_reference(args, world, rank)
         elif args.gemm:
             run_gemm(args, world, rank, local)
+        elif args.act:
+            run_act(args, world, rank, local)
         else:
             run_ours(args, world, rank, local)
     finally:

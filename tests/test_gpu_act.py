@@ -55,7 +55,7 @@ def _decode_gpu(h, fmt):
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_act_quant_bit_exact(dq, fmt_name, dtype):
     rng = np.random.default_rng(3)
-    T, n = 77, 1280                       # ragged last 256-channel round, odd token count
+    T, n = 77, 1280                       # ragged last 512-channel strip, odd token count
     X = rng.standard_normal((T, n)).astype(np.float32)
     X[:, rng.choice(n, 4, replace=False)] *= 50
     X[5, :] = 0.0                          # an all-zero token row
@@ -104,3 +104,44 @@ def test_act_nonfinite_reported(dq, fmt_name, bad):
         dq.act_quant(X.cuda(), fmt_name)
         assert dq.last_device_error() == 5
     assert dq.last_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt_name", ["NVFP4", "INT4", "MXFP4", "INT8", "MXINT8"])
+def test_act_quant_offset_codes_and_strided_x(dq, fmt_name):
+    """Codes written to a buffer that is only as aligned as the interface requires (4 bytes
+    for the 4-bit formats, 8 for the 8-bit ones: one store per lane is split in two) and X
+    read through a row pitch larger than its width give the same codes as the oracle."""
+    import ctypes
+    from calibration_free_dual_b200 import _lib
+    from calibration_free_dual_b200.api import fmt_of
+    rng = np.random.default_rng(11)
+    T, n, ld = 40, 1536, 1600
+    Xfull = torch.from_numpy(rng.standard_normal((T, ld)).astype(np.float32)).to(torch.bfloat16)
+    Xd = Xfull.cuda()
+    X = Xd[:, :n]
+    c = rng.uniform(0.5, 2.0, n).astype(np.float32)
+    fmt = oracle_format(fmt_name)
+    f = fmt_of(fmt_name)
+    cols = n if fmt.bits == 8 else n // 2
+    off = 8 if fmt.bits == 8 else 4
+    buf = torch.zeros(T * cols + 64, dtype=torch.uint8, device="cuda")
+    base = buf.data_ptr() + off
+    sdt = torch.int16 if fmt.scale == "bf16" else torch.uint8
+    scales = torch.empty((T, n // fmt.block), dtype=sdt, device="cuda")
+    ts = torch.empty((1,), dtype=torch.float32, device="cuda")
+    ws = torch.empty((256,), dtype=torch.uint8, device="cuda")
+    cd = torch.from_numpy(c).cuda()
+    lib = _lib.get()
+    st = lib.dq_act_quant(ctypes.c_void_p(X.data_ptr()), _lib.DQ_BF16, T, n, ld,
+                          ctypes.c_void_p(cd.data_ptr()), f, ctypes.c_void_p(base),
+                          ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(ts.data_ptr()),
+                          ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    raw = buf.cpu().numpy()
+    assert not raw[:off].any() and not raw[off + T * cols:].any()   # nothing outside
+    h = dict(x_packed=raw[off:off + T * cols].reshape(T, cols), scales=scales.cpu().numpy(),
+             tensor_scale=ts.cpu().numpy())
+    ora = ora_act(Xfull.float().numpy()[:, :n], fmt, c)
+    _check(h, ora, fmt)
