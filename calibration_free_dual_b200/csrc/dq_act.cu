@@ -170,6 +170,22 @@ __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int 
   if (bad) atomicOr(A.err_word, ERRBIT_NONFINITE);
 }
 
+// Eight binary32 values -> one word of eight E2M1 codes (RNE, saturating), value k in
+// nibble k (byte k/2, low nibble first)
+__device__ __forceinline__ uint32_t e2m1x8_encode(const float2 (&y)[4]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, %8, %7;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0].x), "f"(y[0].y), "f"(y[1].x), "f"(y[1].y), "f"(y[2].x), "f"(y[2].y),
+        "f"(y[3].x), "f"(y[3].y));
+  return out;
+}
+
 template <int ELEM, int SCALE, int B, bool F32IN>
 __global__ void __launch_bounds__(ACT_WARPS * 32, 3)
 act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
@@ -182,9 +198,17 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
   const int64_t col = ww.col, row0 = ww.row0, row1 = ww.row1;
   const bool valid = col < A.n;
   float s_t = 1.0f;
+  // NVFP4: every E4M3 code's decoded scale fl32(s_t * e) and its reciprocal, per CTA
+  __shared__ float2 tbl[SCALE == SCALE_E4M3 ? 128 : 1];
   if constexpr (SCALE == SCALE_E4M3) {
     s_t = nvfp4_tensor_scale(__uint_as_float(*A.amax_bits));
     if (blockIdx.x == 0 && threadIdx.x == 0 && A.tensor_scale != nullptr) *A.tensor_scale = s_t;
+    if (threadIdx.x < 128) {
+      const uint32_t code = (threadIdx.x == 0 || threadIdx.x == 127) ? 1u : threadIdx.x;
+      const float r = __fmul_rn(s_t, e4m3_decode(code));
+      tbl[threadIdx.x] = make_float2(r, __frcp_rn(r));
+    }
+    __syncthreads();
   }
   const int64_t nb = A.n / B, qpitch = BYTE_CODES ? A.n : A.n / 2;
   // a lane's codes (8 bytes; 16 for the 8-bit formats) go out in one store when the code
@@ -209,18 +233,29 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
     uint32_t code = 0;
     float inv = 0.0f;
     if (a > 0.0f) {
-      const ScaleVal sv = project_scale_direct<SCALE>(__fdiv_rn(a, QMAX), s_t);
+      const ScaleVal sv = project_scale<SCALE>(__fdiv_rn(a, QMAX), s_t, tbl);
       code = sv.code;
       inv = sv.ir;
     }
     const float2 iv = make_float2(inv, inv);
     uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if constexpr (ELEM == ELEM_E2M1) {
+      // four conversions straight into the bytes of one word
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-      float2 q;
-      const uint32_t cb = quant2<ELEM>(mul2(x[p], iv), q);
-      if constexpr (BYTE_CODES) w[p >> 1] |= (cb & 0xFFFFu) << (16 * (p & 1));
-      else w[p >> 2] |= (cb & 0xFFu) << (8 * (p & 3));
+      for (int h = 0; h < 2; ++h) {
+        float2 y[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) y[k] = mul2(x[4 * h + k], iv);
+        w[h] = e2m1x8_encode(y);
+      }
+    } else {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        float2 q;
+        const uint32_t cb = quant2<ELEM>(mul2(x[p], iv), q);
+        if constexpr (BYTE_CODES) w[p >> 1] |= (cb & 0xFFFFu) << (16 * (p & 1));
+        else w[p >> 2] |= (cb & 0xFFu) << (8 * (p & 3));
+      }
     }
     if (valid) {
       if (a == 0.0f) w[0] = w[1] = w[2] = w[3] = 0u;   // all-zero block: code 0 (also -0)
