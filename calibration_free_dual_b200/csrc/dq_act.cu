@@ -96,14 +96,6 @@ __device__ __forceinline__ void rescale_chunk(const Chunk<F32IN>& d, const float
   }
 }
 
-// max that propagates NaN (a NaN operand gives NaN): the running |x| maximum of a block is
-// non-finite exactly when one of its elements is, so one test per block suffices
-__device__ __forceinline__ float max_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
-  return d;
-}
-
 __device__ __forceinline__ float absmax16(const float2 (&x)[8]) {
   float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll

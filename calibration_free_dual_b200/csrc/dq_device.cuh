@@ -235,6 +235,14 @@ __device__ __forceinline__ float nvfp4_tensor_scale(float amax) {
   return (amax > 0.0f) ? __fdiv_rn(amax, NVFP4_TENSOR_DIV) : 1.0f;
 }
 
+// max that propagates NaN (a NaN operand gives NaN): a running |x| maximum is non-finite
+// exactly when one of its inputs is, so one test per block or row piece suffices
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
 // ------------------------------------------------------------------ packed fp32x2 math
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }

@@ -101,13 +101,6 @@ __device__ __forceinline__ void load_global(const char* p, bool wide, Raw<ESZ>& 
   }
 }
 
-__device__ __forceinline__ bool nonfinite8(const float2 (&w)[8]) {
-  bool bad = false;
-#pragma unroll
-  for (int p = 0; p < 8; ++p) bad |= !isfinite(w[p].x) | !isfinite(w[p].y);
-  return bad;
-}
-
 // Butterfly reduction of 32 values over the 32/S lanes sharing piece s = lane % S.
 // Lane L ends with the S totals of indices [L - s, L - s + S) (fixed order).
 template <int S>
@@ -338,7 +331,11 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     fetch(0, buf);
     ScaleVal scn;
     if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
-    for (int k = 0; k < RPT; ++k) {
+    // one row step; NEXT: which source the next row comes from (0: none, this is the last
+    // row; 1: shared memory; 2: L2, or zeros past the last row), fixed per loop below so the
+    // row steps carry no per-row test of the source
+    auto step = [&](const int k, auto next_tag) {
+      constexpr int NEXT = decltype(next_tag)::value;
       const int row = g + k * NG;
       float2 w[8];
       unpack<ESZ>(buf, w);
@@ -348,15 +345,26 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         sc = scn;
         old_code = sc.code;
       }
-      if (k + 1 < RPT) {
-        fetch(k + 1, buf);
-        if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+      if constexpr (NEXT == 1) {
+#pragma unroll
+        for (int h = 0; h < ESZ; ++h) {
+          const uint4 v = smp[ESZ * NT * (k + 1) + (h ^ sw)];
+          buf.u[4 * h + 0] = v.x;
+          buf.u[4 * h + 1] = v.y;
+          buf.u[4 * h + 2] = v.z;
+          buf.u[4 * h + 3] = v.w;
+        }
+      } else if constexpr (NEXT == 2) {
+        if (g + (k + 1) * NG < m) load_global<ESZ>(gp + (k + 1) * gstep, wide, buf);
+        else zero<ESZ>(buf);
       }
+      if constexpr (!INIT && NEXT != 0) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
       if constexpr (INIT) {
-        bad |= nonfinite8(w);
+        // NaN-propagating maximum: a is non-finite exactly when one of the piece's values is
         float a = 0.0f;
 #pragma unroll
-        for (int p = 0; p < 8; ++p) a = fmaxf(a, fmaxf(fabsf(w[p].x), fabsf(w[p].y)));
+        for (int p = 0; p < 8; ++p) a = max_nan(a, max_nan(fabsf(w[p].x), fabsf(w[p].y)));
+        bad |= !isfinite(a);
 #pragma unroll
         for (int off = 1; off < LPB; off <<= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
         float v;
@@ -473,7 +481,15 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
           }
         }
       }
-    }
+    };
+    using N0 = std::integral_constant<int, 0>;
+    using N1 = std::integral_constant<int, 1>;
+    using N2 = std::integral_constant<int, 2>;
+    const int kres = min(KS, RPT) - 1;     // row steps whose next row is resident
+    int k = 0;
+    for (; k < kres; ++k) step(k, N1{});
+    for (; k < RPT - 1; ++k) step(k, N2{});
+    step(RPT - 1, N0{});
     if (INIT && bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
 
     // ---- Q-change sums of this pass: per warp (exact), summed by thread 0 below
