@@ -161,7 +161,8 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   float* icvec = reinterpret_cast<float*>(smem + lay.icvec);
   float* red = reinterpret_cast<float*>(smem + lay.red);
   double* errw = reinterpret_cast<double*>(smem + lay.cols);   // [S] per-warp error sums
-  double* wsqw = errw + 8;                                     // [S] per-warp ||W||^2 sums
+  double* e0w = errw + 8;                                      // [NWARP] iteration-0 errors
+  double* wsqw = e0w + NWARP;                                  // [NWARP] ||W||^2 sums
   void* pcodes_v = smem + lay.pcodes;                          // Q-change: previous codes
   float* picvec = reinterpret_cast<float*>(smem + lay.picvec); // Q-change: previous 1/c
   double* qred = reinterpret_cast<double*>(smem + lay.qred);   // Q-change: per-warp sums
@@ -308,21 +309,27 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     return tot;
   };
 
-  double Sj = 0.0;          // ||W_j||^2 of column sj*16 + lane (threads tid < 32*S, lane < 16)
+  double wsq_tile = 0.0;    // ||W||^2 of the tile (thread 0)
 
   // One pass over all rows of the tile. INIT: iteration 0 (scales from absmax or r0,
   // c = c0); otherwise one BCD iteration (Q-step, r-step + projection, c-step). EMIT: the
   // returned state is written.
-  auto pass = [&](auto init_tag, auto emit_tag, const int t) {
+  //
+  // FUSE (with INIT): iteration 0 and iteration 1 in one sweep. Iteration 1's Q-step sees the
+  // state of iteration 0, so its codes are iteration 0's: the pass quantizes once, adds the
+  // iteration-0 error sum (W - r q c)^2 directly, then runs iteration 1's r-step and c-step.
+  auto pass = [&](auto init_tag, auto emit_tag, auto fuse_tag, const int t) {
     constexpr bool INIT = decltype(init_tag)::value;
     constexpr bool EMIT = decltype(emit_tag)::value;
-    float2 accN[8], accD[8], accS[INIT ? 8 : 1];
+    constexpr bool FUSE = INIT && decltype(fuse_tag)::value;
+    constexpr bool ITER = !INIT || FUSE;     // the pass runs an iteration's r- and c-steps
+    float2 accN[8], accD[8];
+    float2 accW2 = make_float2(0.f, 0.f), accE0 = make_float2(0.f, 0.f);   // INIT, FUSE
     float2 accQd = make_float2(0.f, 0.f), accQp = make_float2(0.f, 0.f);   // Q-change
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       accN[p] = make_float2(0.f, 0.f);
       accD[p] = make_float2(0.f, 0.f);
-      if constexpr (INIT) accS[p] = make_float2(0.f, 0.f);
     }
     bool bad = false;
 
@@ -336,7 +343,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     // row steps carry no per-row test of the source
     auto step = [&](const int k, auto next_tag) {
       constexpr int NEXT = decltype(next_tag)::value;
-      const int row = g + k * NG;
+      [[maybe_unused]] const int row = g + k * NG;
       float2 w[8];
       unpack<ESZ>(buf, w);
       ScaleVal sc;
@@ -374,11 +381,12 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
           v = (a > 0.0f) ? __fdiv_rn(a, QMAX) : 1.0f;
         }
         sc = project_scale<SCALE>(v, s_t, tbl);
+        old_code = sc.code;
       }
 
       // Q-step on the binary32 quotient fl32(fl32(w * 1/c) * 1/r)
       float2 q[8];
-      uint32_t codes[4] = {0u, 0u, 0u, 0u};
+      [[maybe_unused]] uint32_t codes[4] = {0u, 0u, 0u, 0u};
       const float2 irr = make_float2(sc.ir, sc.ir);
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
@@ -386,6 +394,15 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         if constexpr (EMIT && BYTE_CODES) codes[p >> 1] |= quant2<ELEM>(x, q[p]) << (16 * (p & 1));
         else if constexpr (EMIT) codes[p >> 2] |= quant2<ELEM>(x, q[p]) << (8 * (p & 3));
         else q[p] = quant2_value<ELEM>(x);
+      }
+      if constexpr (FUSE) {
+        // iteration 0's error W - r q c, straight from its state (c: the initial column scales)
+        const float2 nr = make_float2(-sc.r, -sc.r);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+          const float2 e = fma2(mul2(q[p], nr), cc[p], w[p]);
+          accE0 = fma2(e, e, accE0);
+        }
       }
       if constexpr (EXT && !INIT) {
         if (qch && t >= 2) {
@@ -409,7 +426,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         }
       }
 
-      if (!INIT && upd_r) {
+      if (ITER && upd_r) {
         // r-step: least squares over the block, then projection
         if constexpr (SCALE == SCALE_BF16) {
           // INT4's fine bf16 scale grid: block sums in binary64 keep projection decisions
@@ -449,7 +466,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
       if (lib == 0) {
         set_code(k, sc.code);
-        if constexpr (EXT && !INIT) {
+        if constexpr (EXT && ITER) {
           if (qch) set_pcode(k, old_code);
         }
       }
@@ -461,7 +478,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         const float2 qr = mul2(q[p], rr);
         accN[p] = fma2(w[p], qr, accN[p]);
         accD[p] = fma2(qr, qr, accD[p]);
-        if constexpr (INIT) accS[p] = fma2(w[p], w[p], accS[p]);
+        if constexpr (INIT) accW2 = fma2(w[p], w[p], accW2);
       }
 
       if constexpr (EMIT) {
@@ -506,56 +523,70 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       }
     }
 
-    // ---- column sums (iteration 0 first forms ||W_j||^2, kept by its owner thread)
+    // ---- iteration 0: ||W||^2 of the tile and (FUSE) the direct error sum, per warp
     if constexpr (INIT) {
-      float2 zero2[8];
+      double w2 = (double)accW2.x + (double)accW2.y, e0 = (double)accE0.x + (double)accE0.y;
 #pragma unroll
-      for (int p = 0; p < 8; ++p) zero2[p] = make_float2(0.f, 0.f);
-      Sj = column_totals(accS, zero2);
-      __syncthreads();                       // the reduction buffer is reused
+      for (int off = 16; off >= 1; off >>= 1) {
+        w2 += __shfl_xor_sync(FULL, w2, off);
+        if constexpr (FUSE) e0 += __shfl_xor_sync(FULL, e0, off);
+      }
+      if (lane == 0) {
+        wsqw[warp] = w2;
+        if constexpr (FUSE) e0w[warp] = e0;
+      }
     }
+
+    // ---- column sums
     const double nd = column_totals(accN, accD);
 
     // ---- c-step (closed form) and this pass's error terms: warps 0..S-1, lanes 0..15
     if (tid < 32 * S) {
       const double Dj = __shfl_down_sync(FULL, nd, 16);
-      double e = 0.0, q2 = 0.0;
+      double e = 0.0;
       if (lane < 16) {
         const int j = warp * 16 + lane;
         const double Nj = nd;
         float cj = cvec[j];
-        if (!INIT && qch) picvec[j] = icvec[j];   // 1/c of this pass's Q-step
-        if (!INIT && upd_c && Dj > 0.0) {
+        if (ITER && qch) picvec[j] = icvec[j];   // 1/c of this pass's Q-step
+        if (ITER && upd_c && Dj > 0.0) {
           cj = __fdiv_rn(__double2float_rn(Nj), __double2float_rn(Dj));
           cvec[j] = cj;
           icvec[j] = __frcp_rn(cj);
         }
         if (EMIT) M.c[col0 + j] = cj;
+        // this column's part of ||W - W_hat||^2 beyond ||W_j||^2 (added once per tile)
         const double cd = (double)cj;
-        e = Sj - 2.0 * cd * Nj + cd * cd * Dj;
-        if constexpr (INIT) q2 = Sj;
+        e = cd * cd * Dj - 2.0 * cd * Nj;
       }
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        e += __shfl_xor_sync(FULL, e, off);
-        if constexpr (INIT) q2 += __shfl_xor_sync(FULL, q2, off);
-      }
-      if (lane == 0) {
-        errw[warp] = e;
-        if constexpr (INIT) wsqw[warp] = q2;
-      }
+      for (int off = 16; off >= 1; off >>= 1) e += __shfl_xor_sync(FULL, e, off);
+      if (lane == 0) errw[warp] = e;
     }
     __syncthreads();
-    if constexpr (!INIT) load_c();
+    if constexpr (ITER) load_c();
     if (tid == 0) {
-      double e = 0.0, q2 = 0.0;
+      if constexpr (INIT) {
+        double q2 = 0.0;
 #pragma unroll
-      for (int i = 0; i < S; ++i) {
-        e += errw[i];
-        if constexpr (INIT) q2 += wsqw[i];
+        for (int i = 0; i < NWARP; ++i) q2 += wsqw[i];
+        wsq_tile = q2;
+        M.ws_wsq[tile] = q2;
       }
+      double e = wsq_tile;
+#pragma unroll
+      for (int i = 0; i < S; ++i) e += errw[i];
       M.ws_err[(int64_t)t * tiles + tile] = e;
-      if constexpr (INIT) M.ws_wsq[tile] = q2;
+      if constexpr (FUSE) {
+        double e0 = 0.0;
+#pragma unroll
+        for (int i = 0; i < NWARP; ++i) e0 += e0w[i];
+        M.ws_err[tile] = e0;                          // iteration 0
+        if (qch) {
+          M.ws_qch[2 * tile] = 0.0;                   // iteration 0: no change
+          M.ws_qch[2 * tile + 1] = 0.0;
+        }
+      }
       if (qch) {
         double qd = 0.0, qp = 0.0;
 #pragma unroll
@@ -569,12 +600,16 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     }
   };
 
+  using Y = std::true_type;
+  using N = std::false_type;
   if (T == 0) {
-    pass(std::true_type{}, std::true_type{}, 0);
+    pass(Y{}, Y{}, N{}, 0);                  // iteration 0 only
+  } else if (T == 1) {
+    pass(Y{}, Y{}, Y{}, 1);                  // iterations 0 and 1, emitted
   } else {
-    pass(std::true_type{}, std::false_type{}, 0);
-    for (int t = 1; t < T; ++t) pass(std::false_type{}, std::false_type{}, t);
-    pass(std::false_type{}, std::true_type{}, T);
+    pass(Y{}, N{}, Y{}, 1);                  // iterations 0 and 1
+    for (int t = 2; t < T; ++t) pass(N{}, N{}, N{}, t);
+    pass(N{}, Y{}, N{}, T);
   }
 }
 
