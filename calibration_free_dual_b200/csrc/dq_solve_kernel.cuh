@@ -138,6 +138,10 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
   constexpr float QMAX = elem_qmax<ELEM>();
   constexpr bool BYTE_CODES = (ELEM == ELEM_INT8);        // one code byte per element
   static_assert(NBLK * LPB == S && S >= 1 && S <= 8, "tile shape");
+  // code-shape choices by format (measured on the 8B layer set; results do not depend on
+  // them): the three row loops pay for E4M3 (one-lane blocks) and the bf16-scale formats,
+  // whose extra registers cost the E8M0 formats more than the per-row test saves
+  constexpr bool SPLIT_ROWS = (SCALE != SCALE_E8M0);
 
   const int m = L.m, n = L.n, T = L.T, tiles = L.tiles;
   const int tile = blockIdx.x;
@@ -339,8 +343,8 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     ScaleVal scn;
     if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
     // one row step; NEXT: which source the next row comes from (0: none, this is the last
-    // row; 1: shared memory; 2: L2, or zeros past the last row), fixed per loop below so the
-    // row steps carry no per-row test of the source
+    // row; 1: shared memory; 2: L2, or zeros past the last row; 3: tested per row). With
+    // SPLIT_ROWS the source is fixed per loop below, so the row steps carry no per-row test
     auto step = [&](const int k, auto next_tag) {
       constexpr int NEXT = decltype(next_tag)::value;
       [[maybe_unused]] const int row = g + k * NG;
@@ -365,7 +369,14 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         if (g + (k + 1) * NG < m) load_global<ESZ>(gp + (k + 1) * gstep, wide, buf);
         else zero<ESZ>(buf);
       }
-      if constexpr (!INIT && NEXT != 0) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+      if constexpr (NEXT == 3) {
+        if (k + 1 < RPT) {
+          fetch(k + 1, buf);
+          if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+        }
+      } else if constexpr (!INIT && NEXT != 0) {
+        scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+      }
       if constexpr (INIT) {
         // NaN-propagating maximum: a is non-finite exactly when one of the piece's values is
         float a = 0.0f;
@@ -502,11 +513,15 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     using N0 = std::integral_constant<int, 0>;
     using N1 = std::integral_constant<int, 1>;
     using N2 = std::integral_constant<int, 2>;
-    const int kres = min(KS, RPT) - 1;     // row steps whose next row is resident
-    int k = 0;
-    for (; k < kres; ++k) step(k, N1{});
-    for (; k < RPT - 1; ++k) step(k, N2{});
-    step(RPT - 1, N0{});
+    if constexpr (SPLIT_ROWS) {
+      const int kres = min(KS, RPT) - 1;   // row steps whose next row is resident
+      int k = 0;
+      for (; k < kres; ++k) step(k, N1{});
+      for (; k < RPT - 1; ++k) step(k, N2{});
+      step(RPT - 1, N0{});
+    } else {
+      for (int k = 0; k < RPT; ++k) step(k, std::integral_constant<int, 3>{});
+    }
     if (INIT && bad) atomicOr(L.err_word, ERRBIT_NONFINITE);
 
     // ---- Q-change sums of this pass: per warp (exact), summed by thread 0 below
