@@ -109,8 +109,26 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, 
   if (B == 0 || m <= 0 || n <= 0 || n % B || m > (1 << 24)) return false;
   const int LPB = B / 16;
   const int scb = fmt_scale_bytes(kind);
+  // Tile width: at least 16 rows per thread and pass (S doubles while fewer); for multi-lane
+  // blocks (E8M0, bf16 scales) up to 32 rows while the rows that the resident CTAs stream from
+  // L2 every pass (all but the R in shared memory, one CTA per SM) stay within a share of L2.
+  // More rows per pass spread the per-pass column reduction and barriers over more work; a
+  // wider tile keeps fewer rows resident (8B layer set: MXFP4 72.3 -> 69.4 ms per step).
+  auto streamed_bytes = [&](int s) -> int64_t {
+    const SolveSmem b0 = solve_smem((int)m, 0, s, LPB, esize, scb, qch);
+    const int ng = SOLVE_NT / s;
+    const int64_t rb = (int64_t)16 * s * esize;
+    if (b0.total + 128 > SOLVE_SMEM_MAX) return INT64_MAX;
+    const int64_t r = (int64_t)(SOLVE_SMEM_MAX - b0.total - 128) / rb / ng * ng;
+    return std::max<int64_t>(0, m - r) * rb * 148;
+  };
+  constexpr int64_t L2_STREAM_BUDGET = 48ll << 20;
   int S = LPB;
-  while (S < 8 && m * S < (int64_t)16 * SOLVE_NT && n % (32 * S) == 0) S *= 2;
+  while (S < 8 && n % (32 * S) == 0 &&
+         (m * S < (int64_t)16 * SOLVE_NT ||
+          (LPB >= 2 && m * S < (int64_t)32 * SOLVE_NT &&
+           streamed_bytes(2 * S) <= L2_STREAM_BUDGET)))
+    S *= 2;
   const int NG = SOLVE_NT / S;
   const SolveSmem base = solve_smem((int)m, 0, S, LPB, esize, scb, qch);
   if (base.total + 128 > SOLVE_SMEM_MAX) return false;
