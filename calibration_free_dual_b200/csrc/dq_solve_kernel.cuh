@@ -21,7 +21,9 @@
 //     (FMUL2/FFMA2) and the E2M1/E4M3 cvt instructions;
 //   * per pass, the per-column sums N_j, D_j go through a butterfly inside each warp (fp32)
 //     and a fixed binary64 tree across the 16 warps; the warps that own the tree also form
-//     the closed-form c_j and the pass's error terms. Two barriers per pass, no spin-waits.
+//     the closed-form c_j and the pass's error terms. Two barriers per pass, no spin-waits;
+//   * iterations 0 and 1 share the first pass (iteration 1's codes are iteration 0's), so
+//     T iterations take T passes over the tile.
 #pragma once
 
 #include <algorithm>
