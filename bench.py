@@ -179,7 +179,9 @@ def dist_setup(args):
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+        # short enough that ranks waiting on a lost peer end with an error well before any
+        # outer limit; long enough for the per-rank input generation before the first barrier
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=240))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
