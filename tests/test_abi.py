@@ -149,3 +149,31 @@ def test_linear_validation_and_workspace(dq):
                              0x1000, 8, nul, 0, nul) == 1                      # ldx < K
     assert dq.dq_w4a4_linear(0x1000, 1, 8, 128, 128, nul, 0x1000, 0x1000, 0x1000, 8, nv,
                              0x1000, 8, nul, 0, nul) == 4                      # no workspace
+
+
+def test_act_quant_validation_before_cuda(dq):
+    """Every malformed dq_act_quant call is refused on the host, before anything is queued
+    (the pointers below are never dereferenced: each call fails one check)."""
+    f = dq.fmt_of("NVFP4")
+    P = ctypes.c_void_p
+    X, c, xq, sc, ts, ws = P(0x10000), P(0x20000), P(0x30000), P(0x40000), P(0x50000), P(0x60000)
+    nul = None
+    # zero tokens: nothing to do, success without touching any pointer
+    assert dq.dq_act_quant(nul, 1, 0, 128, 128, nul, f, nul, nul, nul, nul, 0, nul) == 0
+    # ldx < n, negative tokens, unknown dtype
+    assert dq.dq_act_quant(X, 1, 8, 128, 64, c, f, xq, sc, ts, ws, 256, nul) == 1
+    assert dq.dq_act_quant(X, 1, -1, 128, 128, c, f, xq, sc, ts, ws, 256, nul) == 1
+    assert dq.dq_act_quant(X, 9, 8, 128, 128, c, f, xq, sc, ts, ws, 256, nul) == 3
+    # NVFP4 needs the tensor-scale output
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, c, f, xq, sc, nul, ws, 256, nul) == 1
+    # X not 16-byte aligned, or a row pitch that is not a multiple of 16 bytes
+    assert dq.dq_act_quant(P(0x10008), 1, 8, 128, 128, c, f, xq, sc, ts, ws, 256, nul) == 1
+    assert dq.dq_act_quant(X, 1, 8, 128, 132, c, f, xq, sc, ts, ws, 256, nul) == 1
+    # c not 16-byte aligned; codes not 4-byte aligned (8 for the 8-bit formats)
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, P(0x20004), f, xq, sc, ts, ws, 256, nul) == 1
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, c, f, P(0x30002), sc, ts, ws, 256, nul) == 1
+    f8 = dq.fmt_of("MXINT8")
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, c, f8, P(0x30004), sc, ts, ws, 256, nul) == 1
+    # missing or short workspace
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, c, f, xq, sc, ts, nul, 256, nul) == 4
+    assert dq.dq_act_quant(X, 1, 8, 128, 128, c, f, xq, sc, ts, ws, 3, nul) == 4
