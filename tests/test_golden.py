@@ -5,9 +5,10 @@ definition (DualQuant abstract: closed-form block updates of W ~ diag(r) Q diag(
 acceptodds.com abstract: black-box quantizer, scales projected after every update; Figure 1
 (b): iteration 0 is single-scale round-to-nearest; Figure 2 (b): the normalised-MSE trace).
 Each example exercises the format's element ties, its scale projection, both closed forms
-and the trace with exact dyadic numbers. The oracle is checked against them on the CPU with
-4-column blocks; the CUDA path against the same numbers with every row padded by zero
-columns to the format's real block length (zeros change no block maximum or sum).
+and the trace with exact dyadic numbers (INT4, MXFP4, NVFP4, MXINT4 and the 8-bit INT8).
+The oracle is checked against all of them on the CPU with 4-column blocks; the CUDA path
+against the INT4, MXFP4 and NVFP4 ones with every row padded by zero columns to the format's
+real block length (zeros change no block maximum or sum).
 """
 import os
 from fractions import Fraction
@@ -68,7 +69,7 @@ def _bits32(x):
 
 def test_fixture_is_consistent():
     """The fixture's own arithmetic: W has 2 rows of 4; every example is complete."""
-    assert set(EXAMPLES) == {"INT4", "MXFP4", "NVFP4"}
+    assert set(EXAMPLES) == {"INT4", "MXFP4", "NVFP4", "MXINT4", "INT8"}
     for ex in EXAMPLES.values():
         assert len(ex["W"]) == 2 and all(len(r) == 4 for r in ex["W"])
         for k in ("r0_codes", "q0", "mse0", "r1_codes", "N1", "D1", "c1_bits", "mse1"):
@@ -119,7 +120,7 @@ def _padded(ex):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", sorted(EXAMPLES))
+@pytest.mark.parametrize("name", ["INT4", "MXFP4", "NVFP4"])
 def test_cuda_path_reproduces_the_hand_example(name):
     import torch
     import calibration_free_dual_b200 as dq
