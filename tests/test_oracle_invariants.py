@@ -215,3 +215,18 @@ def test_act_quant_blocks_and_zero_blocks(kind):
     nz = a > 0
     ratio = a[nz] / out["d"][nz]
     assert np.all(ratio <= fmt.qmax * 1.5 + 1e-6) and np.all(ratio >= fmt.qmax / 2.1)
+
+
+def test_sqnr_and_dequant_closed_forms():
+    """SQNR = 10 log10(sum x^2 / sum (x - x_hat)^2): a reconstruction scaled by (1 - e) has
+    SQNR -20 log10(e); exact reconstruction is infinite, a zero one is 0 dB. dequant puts the
+    block scale d on each of the block's B elements."""
+    from oracle.actquant import dequant, sqnr
+    x = np.random.default_rng(21).standard_normal((4, 32))
+    for e in (0.5, 0.1, 1e-3):
+        assert sqnr(x, x * (1 - e)) == pytest.approx(-20 * np.log10(e), rel=1e-12)
+    assert sqnr(x, x) == float("inf")
+    assert sqnr(x, np.zeros_like(x)) == pytest.approx(0.0, abs=1e-12)
+    d = np.array([[2.0, 0.5]])
+    q = np.arange(8, dtype=np.float64).reshape(1, 8)
+    np.testing.assert_array_equal(dequant(d, q, 4), [[0, 2, 4, 6, 2, 2.5, 3, 3.5]])
