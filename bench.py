@@ -7,6 +7,10 @@ activation with the column scales of that step's block-0 k_proj (dq_act_quant).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+Other measurements (same JSON conventions): --fmt/--update/--qchange (other formats and the
+ablation modes of the same step), --act (the activation rescale + quantization alone, NVFP4
+and INT4 g=128, against the HBM roofline), --gemm (the W4A4 GEMM consumer).
+
 Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank solves its own layer set
 (different seeds), no collective on the data path; timing is the max over ranks.
 """
