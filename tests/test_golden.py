@@ -52,7 +52,7 @@ def _load():
                 cur[key] = [[_num(t) for t in row.split()] for row in val.split("|")]
             else:
                 vals = [_num(t) for t in val.split()]
-                cur[key] = vals[0] if len(vals) == 1 and key.startswith(("mse", "s_t")) else vals
+                cur[key] = vals[0] if len(vals) == 1 and key.startswith(("mse", "s_t", "qchange")) else vals
     return ex
 
 
@@ -69,7 +69,7 @@ def _bits32(x):
 
 def test_fixture_is_consistent():
     """The fixture's own arithmetic: W has 2 rows of 4; every example is complete."""
-    assert set(EXAMPLES) == {"INT4", "MXFP4", "NVFP4", "MXINT4", "INT8"}
+    assert set(EXAMPLES) == {"INT4", "MXFP4", "NVFP4", "MXINT4", "INT8", "QCHANGE"}
     for ex in EXAMPLES.values():
         assert len(ex["W"]) == 2 and all(len(r) == 4 for r in ex["W"])
         for k in ("r0_codes", "q0", "mse0", "r1_codes", "N1", "D1", "c1_bits", "mse1"):
@@ -112,6 +112,49 @@ def test_oracle_exact_fit_is_a_fixed_point():
     assert out["mse"][1] == 0.0 and out["mse"][2] == 0.0
 
 
+def _qchange_variants(q_prev, q_now, fmt):
+    """qchange[t]^2 by the definition and by three plausible mistakes: normalising by the new
+    iterate, using element codes instead of values, and forgetting the square root."""
+    d = float(np.sum((q_now - q_prev) ** 2))
+    right = d / float(np.sum(q_prev ** 2))
+    cp = F.round_elem(q_prev.astype(np.float32), fmt)[0].astype(np.float64)
+    cn = F.round_elem(q_now.astype(np.float32), fmt)[0].astype(np.float64)
+    return right, {"new-iterate norm": d / float(np.sum(q_now ** 2)),
+                   "codes": float(np.sum((cn - cp) ** 2)) / float(np.sum(cp ** 2)),
+                   "unrooted": right ** 2}
+
+
+def test_oracle_qchange_is_the_hand_value():
+    """Figure 2 (a)'s relative change of Q-hat on the hand example whose W[1, 0] code moves
+    between iterations 1 and 2: qchange = [0, 0, sqrt(1/429)] exactly, with the hand state of
+    the second iteration (codes, r-step, c-step sums, c bits, MSE)."""
+    ex = EXAMPLES["QCHANGE"]
+    fmt = F.make_format(ex["fmt"], 4)
+    W = _arr(ex["W"])
+    out = S.solve(W, fmt, 2)
+    np.testing.assert_array_equal(out["q"], _arr(ex["q2"]))
+    assert [int(v) for v in out["r_codes"][:, 0]] == ex["r2_codes"]
+    N, D = S.c_step_sums(W, _arr(ex["q2"]), out["r"], 4)
+    assert [Fraction(v) for v in N] == ex["N2"]
+    assert [Fraction(v) for v in D] == ex["D2"]
+    assert _bits32(out["c"]) == ex["c2_bits"]
+    assert out["mse"][2] == pytest.approx(float(ex["mse2"]), rel=1e-12)
+    qc = out["qchange"]
+    assert qc[0] == 0.0 and qc[1] == 0.0
+    assert qc[2] ** 2 == pytest.approx(float(ex["qchange2_sq"]), rel=1e-14)
+    assert qc[2] == pytest.approx(float(ex["qchange2_sq"]) ** 0.5, rel=1e-15)
+
+
+def test_qchange_pin_separates_the_plausible_mistakes():
+    """The pinned value tells the definition apart from each mistake the oracle could make."""
+    ex = EXAMPLES["QCHANGE"]
+    fmt = F.make_format(ex["fmt"], 4)
+    right, wrong = _qchange_variants(_arr(ex["q0"]), _arr(ex["q2"]), fmt)
+    assert right == pytest.approx(float(ex["qchange2_sq"]), rel=1e-15)
+    for name, v in wrong.items():
+        assert abs(v - right) > 0.01 * right, name
+
+
 def _padded(ex):
     B = REAL_BLOCK[ex["fmt"]]
     W = np.zeros((2, B), dtype=np.float64)
@@ -150,3 +193,25 @@ def test_cuda_path_reproduces_the_hand_example(name):
             assert abs(mse[1] - float(ex["mse1"])) <= max(1e-4 * float(ex["mse1"]), 1e-6)
         if "s_t" in ex:
             assert out["tensor_scale"].cpu().numpy()[0] == np.float32(float(ex["s_t"]))
+
+
+@pytest.mark.gpu
+def test_cuda_qchange_trace_is_the_hand_value():
+    """The CUDA path's Q-change trace (dq_solve_batched_ex) on the hand example padded to the
+    real MXFP4 block: [0, 0, sqrt(1/429)] (both of its sums are exact), the codes of the
+    second iteration, and the other outputs unchanged by asking for the trace."""
+    import torch
+    import calibration_free_dual_b200 as dq
+
+    ex = EXAMPLES["QCHANGE"]
+    W = torch.from_numpy(_padded(ex).astype(np.float32)).cuda()
+    fmt = F.make_format(ex["fmt"], REAL_BLOCK[ex["fmt"]])
+    out = dq.solve_batched([W], ex["fmt"], 2, qchange=True)[0]
+    torch.cuda.synchronize()
+    assert dq.last_device_error() == 0
+    qc = out["qchange"].cpu().numpy()
+    assert qc[0] == 0.0 and qc[1] == 0.0
+    assert qc[2] == pytest.approx(float(ex["qchange2_sq"]) ** 0.5, rel=1e-15)
+    q = F.decode_elem(F.unpack_codes(out["q_packed"].cpu().numpy()), fmt)
+    np.testing.assert_array_equal(q[:, :4], _arr(ex["q2"]))
+    assert _bits32(out["c"].cpu().numpy()[:4]) == ex["c2_bits"]
