@@ -25,3 +25,17 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # the parity comparisons' agreement figures, when asked for (DQ_PARITY_REPORT=<path>)
+    path = os.environ.get("DQ_PARITY_REPORT")
+    if not path:
+        return
+    try:
+        from tests import _parity
+    except Exception:  # pragma: no cover
+        return
+    import json
+    with open(path, "w") as fh:
+        json.dump(_parity.REPORTS, fh, indent=1)

@@ -13,7 +13,8 @@ import torch
 
 from oracle import formats as F
 from oracle import solver as S
-from tests._parity import compare_solve, assert_monotone, oracle_format, to_host
+from tests._parity import (compare_solve, assert_monotone, oracle_format, oracle_solve,
+                           to_host, torch_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,8 +50,10 @@ def test_single_side_update_matches_oracle(dq, fmt_name, update):
     W = _matrix(77, 384, 512)
     fmt = oracle_format(fmt_name)
     h = _solve(dq, W, fmt_name, 10, update=update)
-    ora = S.solve(W.float().numpy().astype(np.float64), fmt, 10, update=update)
-    compare_solve(h, ora, fmt, label=f"{fmt_name}/{update}")
+    h_prev = _solve(dq, W, fmt_name, 9, update=update)
+    Wd = torch_to_f64(W)
+    ora = oracle_solve(Wd, fmt, 10, update=update)
+    compare_solve(h, ora, fmt, W=Wd, h_prev=h_prev, update=update, label=f"{fmt_name}/{update}")
     assert_monotone(h["mse"], label=f"{fmt_name}/{update}")
     if update == "row":
         np.testing.assert_array_equal(h["c"], np.ones(512, np.float32))

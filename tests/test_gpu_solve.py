@@ -9,7 +9,8 @@ import torch
 
 import workloads as wl
 from oracle import solver as S
-from tests._parity import (oracle_format, to_host, compare_solve, assert_monotone)
+from tests._parity import (oracle_format, to_host, compare_solve, assert_monotone,
+                           oracle_solve, torch_to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -43,6 +44,17 @@ def _run(dq, Wt, fmt_name, iters, r0=None, c0=None):
     return to_host(out)
 
 
+def _check(dq, Wt, fmt_name, iters, label, r0=None, c0=None, **ora_kw):
+    """GPU solve of T and T - 1 iterations against the oracle's solve with its history."""
+    fmt = oracle_format(fmt_name)
+    h = _run(dq, Wt, fmt_name, iters, r0=r0, c0=c0)
+    h_prev = _run(dq, Wt, fmt_name, iters - 1, r0=r0, c0=c0) if iters >= 1 else None
+    Wd = torch_to_f64(Wt)
+    ora = oracle_solve(Wd, fmt, iters, r0=r0, c0=c0, **ora_kw)
+    rep = compare_solve(h, ora, fmt, W=Wd, h_prev=h_prev, label=label)
+    return h, ora, rep
+
+
 CASES = [
     # fmt, dtype, m, n, iters
     ("INT4", "f32", 512, 512, 20),          # the 512x512 fp32 configuration's shape
@@ -71,12 +83,9 @@ CASES = [
 @pytest.mark.parametrize("fmt_name,dtype,m,n,iters", CASES)
 def test_solve_matches_oracle(dq, fmt_name, dtype, m, n, iters):
     W = _matrix(1000 + m + n, m, n, dtype)
-    h = _run(dq, W, fmt_name, iters)
-    fmt = oracle_format(fmt_name)
-    ora = S.solve(W.float().numpy().astype(np.float64), fmt, iters)
-    if fmt.kind == "NVFP4":
+    h, ora, _ = _check(dq, W, fmt_name, iters, f"{fmt_name}/{dtype}/{m}x{n}")
+    if oracle_format(fmt_name).kind == "NVFP4":
         assert np.float32(h["tensor_scale"][0]) == ora["s_t"]
-    compare_solve(h, ora, fmt, label=f"{fmt_name}/{dtype}/{m}x{n}")
     assert_monotone(h["mse"], label=fmt_name)
     assert h["mse"][-1] <= h["mse"][0]
 
@@ -99,17 +108,13 @@ def test_l2_streamed_rows_both_load_widths(dq, fmt_name, m, n):
     hp = to_host(out)
     for key in ("q_packed", "r", "c", "block_scales", "mse"):
         np.testing.assert_array_equal(hp[key], h[key], err_msg=key)
-    fmt = oracle_format(fmt_name)
-    ora = S.solve(W.float().numpy().astype(np.float64), fmt, 8)
-    compare_solve(h, ora, fmt, label=f"{fmt_name}/{m}x{n}/streamed")
+    _check(dq, W, fmt_name, 8, f"{fmt_name}/{m}x{n}/streamed")
 
 
 def test_config1_tile_full(dq):
     cfg = wl.CONFIGS[1]
     W = wl.weight_host(cfg, 0, 0)
-    h = _run(dq, W, "INT4", cfg.iters)
-    ora = S.solve(W.numpy().astype(np.float64), oracle_format("INT4"), cfg.iters)
-    rep = compare_solve(h, ora, oracle_format("INT4"), label="config1")
+    h, ora, rep = _check(dq, W, "INT4", cfg.iters, "config1")
     assert h["mse"][0] / h["mse"][-1] > 4.0, rep
 
 
@@ -138,9 +143,7 @@ def test_warm_start_q_step_is_bit_exact(dq, fmt_name):
     o0 = S.solve(Wd, fmt, 0, r0=ora5["r"], c0=ora5["c"], amax=amax)
     compare_solve(h0, o0, fmt, exact=True, label="warm0")
     np.testing.assert_array_equal(h0["c"], ora5["c"])
-    h1 = _run(dq, W, fmt_name, 1, r0=ora5["r"], c0=ora5["c"])
-    o1 = S.solve(Wd, fmt, 1, r0=ora5["r"], c0=ora5["c"])
-    rep = compare_solve(h1, o1, fmt, label="warm1")
+    h1, o1, rep = _check(dq, W, fmt_name, 1, "warm1", r0=ora5["r"], c0=ora5["c"])
     assert rep["code_match"] == 1.0                        # the Q-step itself is exact
     assert rep["c_rel"] < 1e-6
 
@@ -161,10 +164,12 @@ def test_batched_mixed_shapes(dq):
     shapes = [(256, 512), (128, 512), (256, 512), (64, 1024)]
     Ws = [_matrix(40 + i, m, n, "bf16") for i, (m, n) in enumerate(shapes)]
     outs = dq.solve_batched([w.cuda() for w in Ws], "MXFP4", 6)
+    prev = dq.solve_batched([w.cuda() for w in Ws], "MXFP4", 5)
     fmt = oracle_format("MXFP4")
-    for W, o in zip(Ws, outs):
-        ora = S.solve(W.float().numpy().astype(np.float64), fmt, 6)
-        compare_solve(to_host(o), ora, fmt, label=str(W.shape))
+    for W, o, op in zip(Ws, outs, prev):
+        Wd = torch_to_f64(W)
+        compare_solve(to_host(o), oracle_solve(Wd, fmt, 6), fmt, W=Wd, h_prev=to_host(op),
+                      label=str(W.shape))
 
 
 def test_zero_matrix_rows_and_columns(dq):
@@ -173,9 +178,7 @@ def test_zero_matrix_rows_and_columns(dq):
     W[:, 17] = 0
     W[40:48, 32:64] = 0
     for fmt_name in ["NVFP4", "MXINT4"]:
-        h = _run(dq, W, fmt_name, 6)
-        ora = S.solve(W.float().numpy().astype(np.float64), oracle_format(fmt_name), 6)
-        compare_solve(h, ora, oracle_format(fmt_name), label="zeros")
+        h, _, _ = _check(dq, W, fmt_name, 6, "zeros")
         assert h["c"][17] == 1.0              # an all-zero column keeps its scale
     Z = torch.zeros(64, 64, dtype=torch.bfloat16)
     h = _run(dq, Z, "NVFP4", 3)
