@@ -157,10 +157,16 @@ DQ_API dq_status dq_solve(const void* W, int32_t dtype, int64_t m, int64_t n, in
  * allow a library to call cudaMalloc or any other allocating routine). The DualQuant pages
  * have no counterpart to this call; it exists only for such callers.
  * Same arguments, semantics and outputs as dq_solve, minus workspace and workspace_bytes.
- * Scratch: a fixed DQ_NOALLOC_SCRATCH_BYTES array inside libdq.so (held by every device
- * that loads the library, until the process exits). The first call on a device looks up
- * that array's device address (cudaGetSymbolAddress) with the device current; make that
- * first call before any stream capture. The call allocates and frees nothing.
+ * Scratch: a fixed DQ_NOALLOC_SCRATCH_BYTES array inside libdq.so, held by every device
+ * that loads it until the process exits. The driver places it in device memory when the
+ * array's code module loads: at process start under CUDA_MODULE_LOADING=EAGER, otherwise
+ * (lazy loading, the default) during the first call on the device. A host that hands all
+ * device memory to its own pool should therefore make one call before doing so; once the
+ * pool owns every byte, that first call fails with DQ_ERR_CUDA. The first call in each CUDA
+ * context looks up the array's device address (cudaGetSymbolAddress) in that context and
+ * keeps it for the context (keyed by the context's id, so a context created after a device
+ * reset, or a second context on the device, looks it up afresh); make that first call before
+ * any stream capture. The call allocates and frees nothing.
  * Every call on a device shares the one array and leaves its contents behind; the call
  * clears what must start at zero itself. Calls whose GPU work overlaps (different streams,
  * or different host threads, on the same device) race on the array: serialise them.
