@@ -193,10 +193,12 @@ __device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const floa
 
 // Projection of the least-squares scale num/den inside a BCD iteration. The quotient is a
 // binary32 approximation (its summands are binary32 sums already): fast division, and for
-// E4M3 the scaled quotient num / (den * s_t) directly.
+// E4M3 the scaled quotient num / (den * s_t) directly. An empty block (den = 0: every code
+// of the block is 0) keeps `old_code`; the code is selected first and decoded once, with no
+// branch around the projection.
 template <int SCALE>
 __device__ __forceinline__ ScaleVal project_scale_ls(float num, float den, float s_t,
-                                                     const float2* tbl) {
+                                                     const float2* tbl, uint32_t old_code) {
   uint32_t code;
   if constexpr (SCALE == SCALE_BF16) {
     const float v = __fdividef(num, den);
@@ -210,8 +212,9 @@ __device__ __forceinline__ ScaleVal project_scale_ls(float num, float den, float
     const float u = __fdividef(num, __fmul_rn(den, s_t));
     uint16_t out;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(u));
-    code = max((uint32_t)out, 1u);
+    code = max((uint32_t)(out & 0xFFu), 1u);
   }
+  code = (den > 0.0f) ? code : old_code;
   return scale_decode<SCALE>(code, tbl);
 }
 
@@ -228,6 +231,23 @@ __device__ __forceinline__ ScaleVal project_scale_direct(float v, float s_t) {
   } else {
     return project_scale<SCALE>(v, s_t, nullptr);
   }
+}
+
+// Correctly rounded a / Q for the grid maxima Q = 6, 7, 127 and finite a >= 0, in three
+// operations: q0 = fl32(a * y) with y = fl32(1/Q), the exact residual r = a - q0*Q by one
+// fma, and q1 = fl32(q0 + r*y) by another (the one-step correction of P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990). Checked against binary64 division over every positive binary32: exact
+// for Q = 7 and 127, and for Q = 6 whenever a >= 2^-125; below that (quotients in the
+// subnormal range) the IEEE division is used.
+template <int Q>
+__device__ __forceinline__ float div_qmax(float a) {
+  static_assert(Q == 6 || Q == 7 || Q == 127, "verified divisors only");
+  constexpr float y = 1.0f / (float)Q;
+  if (Q == 6 && a < 0x1p-125f) return __fdiv_rn(a, (float)Q);
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-q0, (float)Q, a);
+  return __fmaf_rn(r, y, q0);
 }
 
 // NVFP4 per-tensor scale from the amax bit pattern.

@@ -109,11 +109,11 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, 
   if (B == 0 || m <= 0 || n <= 0 || n % B || m > (1 << 24)) return false;
   const int LPB = B / 16;
   const int scb = fmt_scale_bytes(kind);
-  // Tile width: at least 16 rows per thread and pass (S doubles while fewer); for multi-lane
-  // blocks (E8M0, bf16 scales) up to 32 rows while the rows that the resident CTAs stream from
-  // L2 every pass (all but the R in shared memory, one CTA per SM) stay within a share of L2.
-  // More rows per pass spread the per-pass column reduction and barriers over more work; a
-  // wider tile keeps fewer rows resident (8B layer set: MXFP4 72.3 -> 69.4 ms per step).
+  // Tile width: at least 16 rows per thread and pass (S doubles while fewer), and up to 32
+  // while the rows that the resident CTAs stream from L2 every pass (all but the R in shared
+  // memory, one CTA per SM) stay within a share of L2. More rows per pass spread the per-pass
+  // column reduction and barriers over more work; a wider tile keeps fewer rows resident
+  // (8B layer set: MXFP4 72.3 -> 69.4 ms per step, NVFP4 solve kernel -1.1%).
   auto streamed_bytes = [&](int s) -> int64_t {
     const SolveSmem b0 = solve_smem((int)m, 0, s, LPB, esize, scb, qch);
     const int ng = SOLVE_NT / s;
@@ -126,7 +126,7 @@ bool plan_solve(int64_t m, int64_t n, int kind, int group, int esize, bool qch, 
   int S = LPB;
   while (S < 8 && n % (32 * S) == 0 &&
          (m * S < (int64_t)16 * SOLVE_NT ||
-          (LPB >= 2 && m * S < (int64_t)32 * SOLVE_NT &&
+          (m * S < (int64_t)32 * SOLVE_NT &&
            streamed_bytes(2 * S) <= L2_STREAM_BUDGET)))
     S *= 2;
   const int NG = SOLVE_NT / S;

@@ -345,8 +345,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     ScaleVal scn;
     if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
     // one row step; NEXT: which source the next row comes from (0: none, this is the last
-    // row; 1: shared memory; 2: L2, or zeros past the last row; 3: tested per row). With
-    // SPLIT_ROWS the source is fixed per loop below, so the row steps carry no per-row test
+    // row; 1: shared memory; 2: L2, or zeros past the last row; 3: tested per row; 4: L2, a
+    // sweep with every row below m, 256-bit loads). With SPLIT_ROWS the source is fixed per
+    // loop below, so the row steps carry no per-row test
     auto step = [&](const int k, auto next_tag) {
       constexpr int NEXT = decltype(next_tag)::value;
       [[maybe_unused]] const int row = g + k * NG;
@@ -370,6 +371,9 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       } else if constexpr (NEXT == 2) {
         if (g + (k + 1) * NG < m) load_global<ESZ>(gp + (k + 1) * gstep, wide, buf);
         else zero<ESZ>(buf);
+      } else if constexpr (NEXT == 4) {
+#pragma unroll
+        for (int h = 0; h < ESZ / 2; ++h) ldg256_keep(gp + (k + 1) * gstep + 32 * h, buf.u + 8 * h);
       }
       if constexpr (NEXT == 3) {
         if (k + 1 < RPT) {
@@ -474,7 +478,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
             num += __shfl_xor_sync(FULL, num, off);
             den += __shfl_xor_sync(FULL, den, off);
           }
-          if (den > 0.0f) sc = project_scale_ls<SCALE>(num, den, s_t, tbl);
+          sc = project_scale_ls<SCALE>(num, den, s_t, tbl, sc.code);
         }
       }
       if (lib == 0) {
@@ -519,6 +523,11 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       const int kres = min(KS, RPT) - 1;   // row steps whose next row is resident
       int k = 0;
       for (; k < kres; ++k) step(k, N1{});
+      // sweeps up to RPT - 2 lie wholly below m (only the last can be partial): with 32-byte
+      // aligned rows, fetched with no per-row test (-2.9% on the 8B layer set)
+      if (wide) {
+        for (; k < RPT - 2; ++k) step(k, std::integral_constant<int, 4>{});
+      }
       for (; k < RPT - 1; ++k) step(k, N2{});
       step(RPT - 1, N0{});
     } else {
