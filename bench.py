@@ -5,19 +5,27 @@ q/k/v/o/gate/up/down, 6.98e9 bf16 weights, NVFP4, 16 BCD iterations) through
 dq_solve_batched, followed by the activation rescale + NVFP4 quantization of an 8192 x 4096
 activation with the column scales of that step's block-0 k_proj (dq_act_quant).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--split]
+
+The JSON line also carries, measured in the same run on one GPU: the activation quantizer
+alone (NVFP4 and INT4 g=128, L2 flushed, SQNR with and without c), the Llama-3.2-1B-shaped
+MXFP4 and Llama-2-7B-shaped MXINT4 layer sets in their own shapes, and the convergence of
+block 0 of the three layer sets (the Q-change trace and the normalised MSE).
 
 Other measurements (same JSON conventions): --fmt/--update/--qchange (other formats and the
-ablation modes of the same step), --act (the activation rescale + quantization alone, NVFP4
-and INT4 g=128, against the HBM roofline), --gemm (the W4A4 GEMM consumer).
+ablation modes of the headline step), --act (the activation quantizer alone), --gemm (the
+W4A4 GEMM consumer), --cpu-plan (the CPU oracle over the configurations' samples).
 
-Prints one JSON line (rank 0). Multi-GPU (torchrun): every rank solves its own layer set
-(different seeds), no collective on the data path; timing is the max over ranks.
+Multi-GPU (torchrun): by default every rank solves its own layer set (different seeds; weak
+scaling); with --split the ranks share ONE layer set, matrices assigned by element count
+(strong scaling, full-model solve time = the slowest rank). No collective on the data path;
+timing is the max over ranks.
 """
 from __future__ import annotations
 
 import argparse
 import ctypes
+import hashlib
 import json
 import math
 import os
@@ -38,40 +46,44 @@ import workloads as wl  # noqa: E402
 METRIC = "BCD weight elems×iters/s and full-model solve s; % of B200 HBM roofline"
 UNIT = "elem*iter/s"
 CFG_ID = 3
-# FP32 operations per element and BCD iteration in the formulation (FMA counted once):
-# Q-step 2 mul + 1 rounding; r-step q*c, W*qc, (qc)^2; c-step q*r, W*qr, (qr)^2.
-OPS_PER_ELEM_ITER = 9
-# iteration 0 (initialisation): |W| max, Q-step (3), c-step sums (3), W^2
-OPS_PER_ELEM_INIT = 8
-# algorithmic bytes per element and iteration of a per-iteration streaming solve (read W
-# in bf16 + NVFP4 scale state read and write): the HBM-equivalent figure
-HBM_BYTES_PER_ELEM_ITER = 2.125
-
+FMT_SPECS = {"NVFP4": ("NVFP4", 16), "MXFP4": ("MXFP4", 32), "MXINT4": ("MXINT4", 32),
+             "INT4": ("INT4", 128), "INT4_G64": ("INT4", 64), "INT8": ("INT8", 128),
+             "MXINT8": ("MXINT8", 32)}
 
 KERNEL_SOURCES = ("dq_solve.cu", "dq_solve_kernel.cuh", "dq_device.cuh", "dq_internal.h")
-PROFILE = os.path.join(ROOT, "profiles", "solve_kernel_8b_nvfp4_full.md")
+PROFILE_JSON = os.path.join(ROOT, "profiles", "solve_kernel_8b_nvfp4.json")
 
 
-def profiled_traffic_per_elem():
-    """DRAM bytes per weight element per solve from the committed ncu summary, or None when
-    the solve kernel's sources have changed since that capture."""
-    import hashlib
-    if not os.path.exists(PROFILE):
-        return None
+def solve_bytes_per_elem(fmt: str, T: int, esize: int = 2) -> float:
+    """Algorithmic bytes per weight element of one solve-kernel run: W read and the block-scale
+    state read and written at its encoded width in every iteration, the codes written once."""
+    kind, B = FMT_SPECS[fmt]
+    scb = 2 if kind in ("INT4", "INT8") else 1
+    code = 1.0 if kind in ("INT8", "MXINT8") else 0.5
+    return T * (esize + 2.0 * scb / B) + code
+
+
+def prepass_bytes_per_elem(fmt: str, esize: int = 2) -> float:
+    """The NVFP4 tensor-scale pre-pass reads W once; the other formats have none."""
+    return float(esize) if FMT_SPECS[fmt][0] == "NVFP4" else 0.0
+
+
+def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "calibration_free_dual_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
-    vals = {}
-    with open(PROFILE) as fh:
-        for line in fh:
-            if ":" in line and line.strip().split(":")[0] in ("source_sha256_16",
-                                                                "dram_bytes_per_elem_solve"):
-                k, v = line.strip().split(":", 1)
-                vals[k.strip()] = v.strip()
-    if vals.get("source_sha256_16") != h.hexdigest()[:16]:
-        return None
-    return float(vals["dram_bytes_per_elem_solve"])
+    return h.hexdigest()[:16]
+
+
+def profiled_solve_kernel():
+    """The ncu figures of the solve kernel (profiles/solve_kernel_8b_nvfp4.json), or {} when
+    the kernel's sources have changed since that capture."""
+    if not os.path.exists(PROFILE_JSON):
+        return {}
+    with open(PROFILE_JSON) as fh:
+        d = json.load(fh)
+    return d if d.get("source_sha256_16") == kernel_source_hash() else {}
 
 
 def workload_name(count: int, elems: int, T: int, fmt: str = "NVFP4", update: str = "both",
@@ -117,6 +129,13 @@ def parse():
                     help="time the W4A4 GEMM consumer instead: the 7 projections of block 0 "
                          "(solved in NVFP4) against --gemm-tokens activation rows")
     ap.add_argument("--gemm-tokens", type=int, default=8192)
+    ap.add_argument("--split", action="store_true",
+                    help="multi-GPU: split one layer set over the ranks by matrix (strong "
+                         "scaling) instead of one layer set per rank")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the activation, 1B/7B layer-set and convergence records")
+    ap.add_argument("--cpu-plan", action="store_true",
+                    help="run the CPU oracle over the configurations' samples instead")
     ap.add_argument("--act", action="store_true",
                     help="time the activation rescale + quantization alone instead: 8192 x "
                          "4096 bf16 activations with a k_proj's c, NVFP4 and INT4 g=128, L2 "
@@ -213,16 +232,86 @@ _ORACLE_FMT = {"NVFP4": ("NVFP4", 16), "MXFP4": ("MXFP4", 32), "MXINT4": ("MXINT
                "MXINT8": ("MXINT8", 32)}
 
 
-def cpu_sample_solve(W: np.ndarray, amax: float, iters: int, fmt: str = "NVFP4",
-                     update: str = "both"):
-    """Oracle solve of a bounded sample; returns (elem*iter/s, seconds, elements)."""
-    from oracle import formats as F
-    from oracle import solver as S
-    t0 = time.perf_counter()
-    S.solve(W, F.make_format(*_ORACLE_FMT[fmt]), iters, amax=amax if fmt == "NVFP4" else None,
-            update=update)
-    dt = time.perf_counter() - t0
-    return W.size * iters / dt, dt, W.size
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def host_ram_gb() -> float:
+    try:
+        return os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES") / 1e9
+    except (ValueError, OSError, AttributeError):  # pragma: no cover
+        return 16.0
+
+
+def oracle_pool_size(n_tasks: int, gb_per_worker: float = 3.0) -> int:
+    """Workers for the oracle: min(host cores, host RAM / gb_per_worker, tasks)."""
+    return max(1, min(host_cores(), int(host_ram_gb() // gb_per_worker), n_tasks))
+
+
+def run_oracle_tasks(tasks, workers: int) -> dict:
+    """Oracle solves over a pool of `workers` processes (oracle/pool.py, run as its own
+    program: the workers import only NumPy and the oracle, never torch or CUDA)."""
+    from oracle import pool
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "tasks.npz")
+        pool.save_tasks(path, tasks)
+        # one thread per worker process: the pool is the parallelism
+        env = dict(os.environ, OMP_NUM_THREADS="1", OPENBLAS_NUM_THREADS="1",
+                   MKL_NUM_THREADS="1")
+        r = subprocess.run([sys.executable, "-m", "oracle.pool", path, str(workers)],
+                           cwd=ROOT, env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                           text=True, check=True)
+    return json.loads(r.stdout.strip().splitlines()[-1])
+
+
+def oracle_task(W, fmt: str, iters: int, amax=None, update: str = "both"):
+    kind, group = _ORACLE_FMT[fmt]
+    return (W, kind, group, iters, amax if kind == "NVFP4" else None, update)
+
+
+def cpu_sample(mats, fmt: str, iters: int, cols: int, per_matrix: int, update="both"):
+    """The oracle as it stands on the host cores: the first `per_matrix` strips of `cols`
+    columns of each matrix (each solved with its whole matrix's amax), over a process pool."""
+    tasks = []
+    for W in mats:
+        amax = float(np.max(np.abs(W)))
+        for k in range(per_matrix):
+            tasks.append(oracle_task(np.ascontiguousarray(W[:, k * cols:(k + 1) * cols]), fmt,
+                                     iters, amax, update))
+    return run_oracle_tasks(tasks, oracle_pool_size(len(tasks)))
+
+
+def block0_host(cfg):
+    """Block 0 of a layer set drawn on the host (binary64 copies of the bf16 weights)."""
+    return [wl.weight_host(cfg, b, p).float().numpy().astype(np.float64)
+            for b, p, _, _ in cfg.layer_set() if b == 0]
+
+
+CPU_SAMPLE_COLS, CPU_SAMPLE_STRIPS = 64, 2
+
+
+def cpu_baseline_record(fmt: str = "NVFP4", update: str = "both") -> dict:
+    """Bounded sample of the headline workload: block 0's seven projections of the 8B layer
+    set, two 64-column strips each, 16 iterations, over a pool of min(cores, RAM / 3 GB)
+    workers; plus the single-core rate on the 512 x 512 fp32 INT4 tile."""
+    cfg = wl.CONFIGS[CFG_ID]
+    r = cpu_sample(block0_host(cfg), fmt, cfg.iters, CPU_SAMPLE_COLS, CPU_SAMPLE_STRIPS, update)
+    c1 = wl.CONFIGS[1]
+    W1 = wl.weight_host(c1, 0, 0).numpy().astype(np.float64)
+    r1 = run_oracle_tasks([oracle_task(W1, "INT4", c1.iters)], 1)
+    return {"value": r["work"] / r["wall_s"], "unit": UNIT, "cores": r["workers"],
+            "kind": "oracle",
+            "sample": "block 0 of the 8B layer set, 7 projections x %d strips of %d columns "
+                      "(%d oracle solves, %.3g elem*iter), %s, %d iterations, %d worker "
+                      "processes (host: %d cores); %.2f s wall, %.1f s of CPU work"
+                      % (CPU_SAMPLE_STRIPS, CPU_SAMPLE_COLS, r["tasks"], r["work"], fmt,
+                         cfg.iters, r["workers"], host_cores(), r["wall_s"], r["cpu_s"]),
+            "per_core_value": r["work"] / r["cpu_s"],
+            "single_core_512x512_int4": {"value": r1["work"] / r1["wall_s"], "unit": UNIT,
+                                         "seconds": r1["wall_s"]}}
 
 
 def run_reference(args, world, rank):
@@ -230,49 +319,294 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     cfg = wl.CONFIGS[CFG_ID]
-    Wk = wl.weight_host(cfg, 0, 1).float().numpy().astype(np.float64)     # block-0 k_proj
-    amax = float(np.max(np.abs(Wk)))
-    sample = Wk[:, :1024]
-    desc = "block-0 k_proj of the 8B layer set, columns 0..1023 (1024x1024), 16 iterations"
+    mats = block0_host(cfg)
+    desc = ("block 0 of the 8B layer set, 7 projections x %d strips of %d columns, NVFP4, "
+            "16 iterations, over a process pool" % (CPU_SAMPLE_STRIPS, CPU_SAMPLE_COLS))
     for _ in range(args.warmup):
-        cpu_sample_solve(sample, amax, cfg.iters)
-    times = []
+        cpu_sample(mats, "NVFP4", cfg.iters, CPU_SAMPLE_COLS, CPU_SAMPLE_STRIPS)
+    works, walls, P = 0, 0.0, 1
     for _ in range(args.steps):
-        _, dt, _ = cpu_sample_solve(sample, amax, cfg.iters)
-        times.append(dt)
-    tot = sum(times)
-    value = sample.size * cfg.iters * args.steps / tot
+        r = cpu_sample(mats, "NVFP4", cfg.iters, CPU_SAMPLE_COLS, CPU_SAMPLE_STRIPS)
+        works += r["work"]
+        walls += r["wall_s"]
+        P = r["workers"]
+    value = works / walls
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "ms_per_step": 1e3 * walls / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(len(cfg.layer_set()), cfg.elements(), cfg.iters),
                    "sample": desc},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": P, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
+def run_cpu_plan(args):
+    """The CPU baseline plan: the single-core rate on the 512 x 512 tile; the whole 512 x 512
+    tile, 1B layer set and activation workload; blocks {0, L/2, L-1} of the 8B and 7B layer
+    sets (all seven projections), each over a process pool, wall times measured."""
+    from oracle import formats as F
+    from oracle import solver as S
+    from oracle.actquant import act_quant as ora_act
+    out = {"host_cores": host_cores(), "host_ram_gb": round(host_ram_gb(), 1)}
+    t_all = time.perf_counter()
+    c1 = wl.CONFIGS[1]
+    W1 = wl.weight_host(c1, 0, 0).numpy().astype(np.float64)
+    r1 = run_oracle_tasks([oracle_task(W1, "INT4", c1.iters)], 1)
+    out["config1_single_core"] = {"elem_iter_per_s": r1["work"] / r1["wall_s"],
+                                  "seconds": r1["wall_s"]}
+    for cid, sample in ((2, False), (3, True), (4, True)):
+        cfg = wl.CONFIGS[cid]
+        L = cfg.blocks
+        keep = sorted({0, L // 2, L - 1}) if sample else list(range(L))
+        layer = [e for e in cfg.layer_set() if e[0] in keep]
+        tasks = []
+        for b, p, m, n in layer:
+            W = wl.weight_host(cfg, b, p).float().numpy().astype(np.float64)
+            amax = float(np.max(np.abs(W)))
+            for j in range(0, n, 512):
+                tasks.append(oracle_task(np.ascontiguousarray(W[:, j:j + 512]), cfg.fmt.kind,
+                                         cfg.iters, amax))
+        r = run_oracle_tasks(tasks, oracle_pool_size(len(tasks)))
+        elems = sum(m * n for _, _, m, n in layer)
+        rec = {"matrices": len(layer), "elements": elems, "workers": r["workers"],
+               "wall_s": r["wall_s"], "cpu_s": r["cpu_s"],
+               "elem_iter_per_s": r["work"] / r["wall_s"], "measured": True}
+        if sample:
+            rec["blocks"] = keep
+            rec["full_set_wall_s_extrapolated"] = r["wall_s"] * cfg.elements() / elems
+        out["config%d" % cid] = rec
+    # activation workload: its k_proj solve and both quantizations
+    Wk = wl.weight_host(wl.ACT_KPROJ, 0, 1).float().numpy().astype(np.float64)
+    X = wl.act_host().float().numpy()
+    t0 = time.perf_counter()
+    c = S.solve(Wk, F.make_format("MXFP4"), wl.ACT_KPROJ.iters)["c"]
+    for kind, g in (("NVFP4", 16), ("INT4", 128)):
+        ora_act(X, F.make_format(kind, g), c)
+    out["config5"] = {"wall_s": time.perf_counter() - t0, "workers": 1,
+                      "what": "MXFP4 k_proj solve (1024 x 4096, 16 iterations) + NVFP4 and "
+                              "INT4 g=128 quantization of 8192 x 4096"}
+    out["config1_full"] = {"wall_s": out["config1_single_core"]["seconds"], "workers": 1,
+                           "what": "the whole 512 x 512 tile is one solve"}
+    out["total_wall_s"] = time.perf_counter() - t_all
+    print(json.dumps({"cpu_plan": out}), flush=True)
+
+
 # --------------------------------------------------------------------------- our path
+class KernelTimer:
+    """CUDA events recorded by the library around each solve-kernel launch (on the launch
+    stream), for `cap` launches."""
+
+    def __init__(self, lib, stream, cap: int):
+        self.lib, self.cap = lib, cap
+        self.ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+        self.ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+        for e in self.ev_s + self.ev_e:
+            e.record(stream)                    # creates the underlying cudaEvent
+        self.arr_s = (ctypes.c_void_p * cap)(*[e.cuda_event for e in self.ev_s])
+        self.arr_e = (ctypes.c_void_p * cap)(*[e.cuda_event for e in self.ev_e])
+        self.used = 0
+
+    def __enter__(self):
+        self.lib.dq_set_timing_events(self.arr_s, self.arr_e, self.cap)
+        return self
+
+    def __exit__(self, *exc):
+        self.used = self.lib.dq_timing_events_used()
+        self.lib.dq_set_timing_events(None, None, 0)
+
+    def ms(self) -> float:
+        return sum(a.elapsed_time(b) for a, b in zip(self.ev_s[:self.used], self.ev_e[:self.used]))
+
+
+def _mats(Ws, outs):
+    from calibration_free_dual_b200 import _lib
+    arr = (_lib.dq_matrix * len(Ws))()
+    for i, (W, o) in enumerate(zip(Ws, outs)):
+        arr[i] = _lib.dq_matrix(W.data_ptr(), W.shape[0], W.shape[1], W.stride(0), None,
+                                None, o["q_packed"].data_ptr(), o["r"].data_ptr(),
+                                o["c"].data_ptr(), o["block_scales"].data_ptr(),
+                                o["tensor_scale"].data_ptr(), o["mse"].data_ptr())
+    return arr
+
+
+def hbm_roofline(bytes_total: float, ms: float, peaks, peak_src, **extra) -> dict:
+    gbs = bytes_total / (ms * 1e-3) / 1e9 if ms > 0 else None
+    hbm = float(peaks["hbm_gbs"])
+    d = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+         "frac": gbs / hbm if gbs else None,
+         "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_src
+         if peak_src == "measured" else "fallback 6650 GB/s"}
+    d.update(extra)
+    return d
+
+
+def convergence(mse: np.ndarray, qchange: np.ndarray) -> dict:
+    """The pages' convergence figures for one matrix: the relative change of Q-hat at the
+    last iteration (Figure 2 (a)), the first iteration whose normalised-MSE drop is under 1%
+    (Figure 2 (b)), and single-scale over final MSE."""
+    drop = (mse[:-1] - mse[1:]) / np.maximum(mse[:-1], 1e-300)
+    below = [t + 1 for t in range(len(drop)) if drop[t] < 0.01]
+    return {"qchange_last": float(qchange[-1]), "qchange_max": float(np.max(qchange)),
+            "first_iter_drop_below_1pct": below[0] if below else None,
+            "mse0_over_mseT": float(mse[0] / mse[-1]) if mse[-1] > 0 else None}
+
+
+def block0_convergence(dq, cfg, dev, fmt_name) -> dict:
+    """Q-change and MSE traces of block 0 of a layer set (solved once with the trace on)."""
+    layer = [e for e in cfg.layer_set() if e[0] == 0]
+    Ws = [wl.weight_device(cfg, b, p, device=dev) for b, p, _, _ in layer]
+    outs = dq.solve_batched(Ws, fmt_name, cfg.iters, qchange=True)
+    res = {}
+    for (b, p, m, n), o in zip(layer, outs):
+        res[wl.PROJ[p]] = convergence(o["mse"].cpu().numpy(), o["qchange"].cpu().numpy())
+    del Ws, outs
+    return res
+
+
+def time_layer_set(dq, lib, cfg, fmt_name, dev, steps, warmup, rank=0, stream=None):
+    """One dq_solve_batched over a whole layer set per step: (ms per step, solve-kernel ms per
+    step, elements, launches per step)."""
+    from calibration_free_dual_b200 import _lib
+    stream = stream or torch.cuda.current_stream(dev)
+    layer = cfg.layer_set()
+    Ws = [wl.weight_device(cfg, b, p, device=dev, seed_offset=rank) for b, p, _, _ in layer]
+    f = dq.fmt_of(fmt_name)
+    T = cfg.iters
+    outs = [dq.api.solve_outputs(W.shape[0], W.shape[1], f, T, dev) for W in Ws]
+    count = len(Ws)
+    ms_ = (ctypes.c_int64 * count)(*[W.shape[0] for W in Ws])
+    ns_ = (ctypes.c_int64 * count)(*[W.shape[1] for W in Ws])
+    need = lib.dq_solve_workspace_bytes(count, ms_, ns_, f, T)
+    ws = torch.empty((need,), dtype=torch.uint8, device=dev)
+    mats = _mats(Ws, outs)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        st = lib.dq_solve_batched(mats, count, _lib.DQ_BF16, f, T, ctypes.c_void_p(ws.data_ptr()),
+                                  need, sp)
+        if st != 0:
+            raise dq.DQError(st, "dq_solve_batched")
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    per_step = sum((g + 63) // 64 for g in _group_sizes(layer))
+    timer = KernelTimer(lib, stream, per_step * steps)
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with timer:
+        t0.record(stream)
+        for _ in range(steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error while timing %s" % cfg.name)
+    elems = sum(W.numel() for W in Ws)
+    res = (t0.elapsed_time(t1) / steps, timer.ms() / steps, elems, per_step)
+    del Ws, outs, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def config_record(dq, lib, cid, dev, steps, warmup, peaks, peak_src) -> dict:
+    """A layer set in its own shapes and format: throughput, full-model solve seconds, the
+    solve kernel's HBM fraction on the algorithmic bytes, block-0 convergence."""
+    cfg = wl.CONFIGS[cid]
+    fmt_name = cfg.fmt.kind
+    ms, kms, elems, per_step = time_layer_set(dq, lib, cfg, fmt_name, dev, steps, warmup)
+    bpe = solve_bytes_per_elem(fmt_name, cfg.iters)
+    return {"workload": "%s (%d matrices, %.3e bf16 weights), %s, %d BCD iterations"
+                        % (cfg.name, len(cfg.layer_set()), elems, fmt_name, cfg.iters),
+            "value": elems * cfg.iters / (ms * 1e-3), "unit": UNIT,
+            "full_model_solve_s": ms * 1e-3, "solve_kernel_ms": kms,
+            "roofline": hbm_roofline(bpe * elems, kms, peaks, peak_src, kernel="solve_kernel",
+                                     bytes_per_elem=bpe, traffic=None),
+            "convergence_block0": block0_convergence(dq, cfg, dev, fmt_name)}
+
+
+ACT_BYTES_PER_ELEM = {"NVFP4": 2.0 + 0.5 + 1.0 / 16, "INT4": 2.0 + 0.5 + 2.0 / 128}
+
+
+def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dict:
+    """dq_act_quant alone on the activation workload (8192 x 4096 bf16) with column scales c,
+    NVFP4 and INT4 g=128: device time per call with L2 flushed before it, the HBM fraction
+    on the algorithmic bytes, and the SQNR of the decoded activation with and without c."""
+    T, n = X.shape
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)    # 2x the 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    launches = 0
+    for fmt in ("NVFP4", "INT4"):
+        for _ in range(max(warmup, 1)):
+            dq.act_quant(X, fmt, c)
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        barrier(world)
+        l0 = lib.dq_kernel_launches()
+        for e0, e1 in evs:
+            flush.fill_(1)                     # L2 holds none of X when the call starts
+            # a GPU-side wait of ~0.1 ms lets the host enqueue the whole call before e0 is
+            # reached, so the events see the call's device time, not the Python wrapper's
+            torch.cuda._sleep(200_000)
+            e0.record(stream)
+            out = dq.act_quant(X, fmt, c)
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        launches += lib.dq_kernel_launches() - l0
+        if dq.last_device_error() != 0:
+            raise RuntimeError("device error during the activation timing")
+        ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / steps, world)
+        sq = {"with_c": _sqnr(X.float() * c, _act_decode(dq, out, fmt, T, n))}
+        out0 = dq.act_quant(X, fmt, None)
+        sq["without_c"] = _sqnr(X.float(), _act_decode(dq, out0, fmt, T, n))
+        res[fmt] = {"us_per_call": ms * 1e3, "elems_per_s": world * T * n / (ms * 1e-3),
+                    "sqnr_db": sq,
+                    "roofline": hbm_roofline(ACT_BYTES_PER_ELEM[fmt] * T * n, ms, peaks,
+                                             peak_src, bytes_per_elem=ACT_BYTES_PER_ELEM[fmt],
+                                             traffic=None)}
+    del flush
+    return {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) times the "
+                        "step's block-0 k_proj c; L2 flushed (256 MB written) before every "
+                        "call; device time of the call (its launches)",
+            "formats": res, "gpu_launches": int(launches)}
+
+
 def run_ours(args, world, rank, local):
     import calibration_free_dual_b200 as dq
     from calibration_free_dual_b200 import _lib
+    from calibration_free_dual_b200.shard import assign, loads
 
     dev = torch.device("cuda", local)
     cfg = wl.CONFIGS[CFG_ID]
-    layer = cfg.layer_set()
+    full_layer = cfg.layer_set()
     if args.blocks is not None:
-        layer = [e for e in layer if e[0] < args.blocks]
+        full_layer = [e for e in full_layer if e[0] < args.blocks]
     T = cfg.iters
     fmt = dq.fmt_of(args.fmt)
     headline = args.fmt == "NVFP4" and args.update == "both" and not args.qchange
     stream = torch.cuda.current_stream(dev)
+    split = args.split and world > 1
+    if split:
+        # one layer set shared by the ranks, matrices assigned by element count
+        sizes = [m * n for _, _, m, n in full_layer]
+        parts = assign(sizes, world)
+        layer = [full_layer[i] for i in parts[rank]]
+        seed_offset = 0
+    else:
+        layer = full_layer
+        seed_offset = rank
 
     # inputs (device-generated, seeded per rank) and preallocated outputs
-    Ws = [wl.weight_device(cfg, b, p, device=dev, seed_offset=rank) for b, p, _, _ in layer]
+    Ws = [wl.weight_device(cfg, b, p, device=dev, seed_offset=seed_offset)
+          for b, p, _, _ in layer]
     X = wl.act_device(device=dev)
     outs = [dq.api.solve_outputs(W.shape[0], W.shape[1], fmt, T, dev) for W in Ws]
     count = len(Ws)
@@ -291,24 +625,21 @@ def run_ours(args, world, rank, local):
     act_proto = dq.api.solve_outputs(X.shape[0], X.shape[1], fmt, 0, dev)
     act_out = dict(x_packed=act_proto["q_packed"], scales=act_proto["block_scales"],
                    tensor_scale=act_proto["tensor_scale"])
-    act_ws = torch.empty((256,), dtype=torch.uint8, device=dev)
-    k0 = next(i for i, (b, p, _, _) in enumerate(layer) if b == 0 and p == 1)
+    act_ws = torch.empty((lib.dq_act_quant_workspace_bytes(X.shape[0], X.shape[1], fmt),),
+                         dtype=torch.uint8, device=dev)
+    # the activation's column scales: this rank's first k_proj (block 0's when it has it)
+    k0 = next((i for i, (b, p, _, _) in enumerate(layer) if p == 1),
+              0 if layer else None)
 
     def mats_for(Wlist, olist=None):
-        olist = outs if olist is None else olist
-        arr = (_lib.dq_matrix * len(Wlist))()
-        for i, (W, o) in enumerate(zip(Wlist, olist)):
-            arr[i] = _lib.dq_matrix(W.data_ptr(), W.shape[0], W.shape[1], W.stride(0), None,
-                                    None, o["q_packed"].data_ptr(), o["r"].data_ptr(),
-                                    o["c"].data_ptr(), o["block_scales"].data_ptr(),
-                                    o["tensor_scale"].data_ptr(), o["mse"].data_ptr())
-        return arr
+        return _mats(Wlist, outs if olist is None else olist)
 
     mats = mats_for(Ws)
-    sptr = ctypes.c_void_p(stream.cuda_stream)
 
     def solve_call(mats_arr, n_mats, strm):
         sp = ctypes.c_void_p(strm.cuda_stream)
+        if n_mats == 0:
+            return
         if opts is None:
             st = lib.dq_solve_batched(mats_arr, n_mats, _lib.DQ_BF16, fmt, T,
                                       ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
@@ -319,11 +650,13 @@ def run_ours(args, world, rank, local):
         if st != 0:
             raise dq.DQError(st, "dq_solve_batched")
 
+    c_act = outs[k0]["c"] if k0 is not None else None
+
     def act_call(Xin, strm):
         st = lib.dq_act_quant(ctypes.c_void_p(Xin.data_ptr()), _lib.DQ_BF16, Xin.shape[0],
                               Xin.shape[1], Xin.stride(0),
-                              ctypes.c_void_p(outs[k0]["c"].data_ptr()), fmt,
-                              ctypes.c_void_p(act_out["x_packed"].data_ptr()),
+                              ctypes.c_void_p(c_act.data_ptr() if c_act is not None else 0),
+                              fmt, ctypes.c_void_p(act_out["x_packed"].data_ptr()),
                               ctypes.c_void_p(act_out["scales"].data_ptr()),
                               ctypes.c_void_p(act_out["tensor_scale"].data_ptr()),
                               ctypes.c_void_p(act_ws.data_ptr()), act_ws.numel(),
@@ -336,6 +669,7 @@ def run_ours(args, world, rank, local):
         act_call(Xin, stream)
 
     elems = sum(W.numel() for W in Ws)
+    elems_job = sum(m * n for _, _, m, n in full_layer) if split else world * elems
     for _ in range(args.warmup):
         step(mats, X)
     torch.cuda.synchronize(dev)
@@ -343,14 +677,8 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device error during warm-up")
 
     # per-launch events for the solve kernel over the timed region
-    per_step = sum((n + 63) // 64 for n in _group_sizes(layer))   # launches per step
-    cap = per_step * args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
-    for e in ev_s + ev_e:
-        e.record(stream)                    # creates the underlying cudaEvent
-    arr_s = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_s])
-    arr_e = (ctypes.c_void_p * cap)(*[e.cuda_event for e in ev_e])
+    per_step = sum((g + 63) // 64 for g in _group_sizes(layer))   # launches per step
+    timer = KernelTimer(lib, stream, max(1, per_step * args.steps))
     torch.cuda.synchronize(dev)
 
     clocks = ClockSampler(dev.index)
@@ -359,16 +687,14 @@ def run_ours(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = lib.dq_kernel_launches()
-    lib.dq_set_timing_events(arr_s, arr_e, cap)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step(mats, X)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    used = lib.dq_timing_events_used()
-    lib.dq_set_timing_events(None, None, 0)
+    with timer:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(mats, X)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
     launches = lib.dq_kernel_launches() - launches0
     barrier(world)
     clk = clocks.stop()
@@ -376,68 +702,96 @@ def run_ours(args, world, rank, local):
     ms_total = reduce_max(ms_total, world)
     if dq.last_device_error() != 0:
         raise RuntimeError("device error during the timed region")
-    kern_ms = sum(a.elapsed_time(b) for a, b in zip(ev_s[:used], ev_e[:used]))
+    kern_ms = timer.ms()
 
     ms_step = ms_total / args.steps
-    value = world * elems * T / (ms_step * 1e-3)
+    value = elems_job * T / (ms_step * 1e-3)
 
     peaks, peak_src = _peaks()
     sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-    alu_peak = 148 * 128 * sm_max * 1e6 / 1e12                         # Tops/s FP32
-    ops = args.steps * elems * (OPS_PER_ELEM_ITER * T + OPS_PER_ELEM_INIT)
-    achieved = ops / (kern_ms * 1e-3) / 1e12 if kern_ms > 0 else None
-    # W in bf16 plus the block-scale state read and written once per iteration
-    scb = 2 if args.fmt.startswith("INT") else 1
-    hbm_bpe = 2.0 + 2.0 * scb / fmt.group
-    hbm_equiv = args.steps * elems * T * hbm_bpe / (kern_ms * 1e-3) / 1e9
-    tpe = profiled_traffic_per_elem() if headline else None
-    traffic = tpe * elems / per_step if tpe is not None else None        # bytes per launch
-    roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tops/s",
-            "frac": achieved / alu_peak if achieved else None, "traffic": traffic,
-            "traffic_unit": "DRAM bytes per solve launch (ncu capture, layer-set average)",
-            "peak_source": "148 SMs x 128 FP32 lanes x %.0f MHz (FMA = 1 op)" % sm_max,
-            "kernel": "solve_kernel", "kernel_ms_per_step": kern_ms / args.steps,
-            "launches_timed": used,
-            "hbm_equivalent": {"bytes_per_elem_iter": hbm_bpe,
-                               "achieved_GBps": hbm_equiv,
-                               "frac_of_hbm_peak": hbm_equiv / float(peaks["hbm_gbs"]),
-                               "peak_GBps": float(peaks["hbm_gbs"]), "peak_source": peak_src}}
+    # the solve kernel against HBM on the algorithmic bytes (W and the block-scale state
+    # every iteration, the codes once): what a per-iteration streaming solve would move
+    bpe = solve_bytes_per_elem(args.fmt, T)
+    prof = profiled_solve_kernel() if headline else {}
+    traffic = None
+    if prof.get("dram_bytes_per_elem_solve") is not None:
+        traffic = prof["dram_bytes_per_elem_solve"] * elems / max(per_step, 1)
+    kms_step = kern_ms / args.steps
+    roof = hbm_roofline(bpe * elems, kms_step, peaks, peak_src, traffic=traffic,
+                        kernel="solve_kernel", bytes_per_elem=bpe,
+                        kernel_ms_per_step=kms_step, launches_timed=timer.used,
+                        traffic_unit="DRAM bytes per solve launch (ncu capture of the same "
+                                     "kernel source, layer-set average), null if the kernel "
+                                     "changed since")
+    act_bpe = ACT_BYTES_PER_ELEM.get(args.fmt if args.fmt != "INT4_G64" else "INT4")
+    act_elems = X.numel()
+    step_bytes = (bpe + prepass_bytes_per_elem(args.fmt)) * elems + (act_bpe or 0) * act_elems
+    roof_step = hbm_roofline(step_bytes, ms_total / args.steps, peaks, peak_src,
+                             bytes_per_elem=bpe + prepass_bytes_per_elem(args.fmt),
+                             includes="solve kernel, NVFP4 tensor-scale pre-pass, trace "
+                                      "finalisation and the activation quantization",
+                             per_gpu=True)
+    issue = None
+    if prof.get("inst_per_elem_pass") is not None:
+        warp_inst = prof["inst_per_elem_pass"] / 32.0 * elems * T
+        ach = warp_inst / (kms_step * 1e-3)
+        pk = 148 * 4 * sm_max * 1e6
+        issue = {"bound": "issue", "inst_per_elem_pass": prof["inst_per_elem_pass"],
+                 "achieved": ach, "peak": pk, "unit": "warp-instructions/s", "frac": ach / pk,
+                 "peak_source": "148 SMs x 4 schedulers x %.0f MHz, one instruction per "
+                                "scheduler per cycle; instruction count from ncu" % sm_max}
 
     # ------------------------------------------------------------------ end to end
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, world, dev, Ws, X, outs, act_out, solve_call, act_call, mats_for,
-                      layer, elems, T)
+                      layer, elems, T, elems_job)
+
+    # ------------------------------------------------------------------ extra records
+    extra = {}
+    if world == 1 and headline and not args.no_extra:
+        extra["act"] = act_record(dq, lib, X, c_act, dev, args.steps, args.warmup, world,
+                                  peaks, peak_src)
+        conv3 = block0_convergence(dq, cfg, dev, "NVFP4")
+        del Ws, outs, mats, ws
+        torch.cuda.empty_cache()
+        extra["configs"] = {"1B_MXFP4": config_record(dq, lib, 2, dev, args.steps,
+                                                      args.warmup, peaks, peak_src),
+                            "7B_MXINT4": config_record(dq, lib, 4, dev, args.steps,
+                                                       args.warmup, peaks, peak_src)}
+        extra["configs"]["8B_NVFP4"] = {"convergence_block0": conv3}
 
     # ------------------------------------------------------------------ CPU baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        Wk = Ws[k0].float().cpu().numpy().astype(np.float64)
-        amax = float(np.max(np.abs(Wk)))
-        v, dt, n_el = cpu_sample_solve(Wk, amax, T, args.fmt, args.update)
-        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "block-0 k_proj (1024x4096) of this layer set, %s, 16 iterations, "
-                         "%.1f s, single process" % (args.fmt, dt)}
+        cpu = cpu_baseline_record(args.fmt, args.update)
 
     if rank == 0:
+        cfgd = {"workload": workload_name(len(full_layer), sum(m * n for _, _, m, n in full_layer),
+                                          T, args.fmt, args.update, args.qchange),
+                "full_model_solve_s": ms_step * 1e-3,
+                "l2": "inputs larger than L2 (%.1f GB of weights per step)" % (elems * 2 / 1e9),
+                "blocks": args.blocks if args.blocks is not None else cfg.blocks}
+        if split:
+            cfgd["parallelism"] = "one layer set split over %d GPUs by matrix" % world
+            cfgd["elements_per_rank"] = loads([m * n for _, _, m, n in full_layer], parts)
+        else:
+            cfgd["parallelism"] = "one layer set per GPU (weak)"
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": workload_name(count, elems, T, args.fmt, args.update,
-                                                 args.qchange),
-                       "full_model_solve_s": ms_step * 1e-3,
-                       "l2": "inputs larger than L2 (%.1f GB of weights per step)"
-                             % (elems * 2 / 1e9),
-                       "parallelism": "one layer set per GPU (weak)",
-                       "blocks": args.blocks if args.blocks is not None else cfg.blocks},
+            "higher_is_better": True, "scaling": "strong" if split else "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": cfgd,
             "roofline": roof,
+            "roofline_step": roof_step,
+            "roofline_issue": issue,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(launches),
             "clocks": clk,
         }
+        line.update(extra)
         print(json.dumps(line), flush=True)
 
 
@@ -453,7 +807,7 @@ def _group_sizes(layer):
 
 
 def run_e2e(args, world, dev, Ws, X, outs, act_out, solve_call, act_call, mats_for, layer,
-            elems, T):
+            elems, T, elems_job):
     """The same step through the public API from pinned host buffers, results read back to
     pinned host buffers, pipelined the way a user streams a model: one dq_solve_batched per
     block of the layer set on the compute stream, while a copy stream brings in the next
@@ -524,7 +878,7 @@ def run_e2e(args, world, dev, Ws, X, outs, act_out, solve_call, act_call, mats_f
     b.record(comp)
     torch.cuda.synchronize(dev)
     ms = reduce_max(a.elapsed_time(b), world) / args.steps
-    return {"value": world * elems * T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+    return {"value": elems_job * T / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "pipeline": "per block: H2D, dq_solve_batched and D2H on three streams"}
 
@@ -661,9 +1015,6 @@ def run_gemm(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-ACT_BYTES_PER_ELEM = {"NVFP4": 2.0 + 0.5 + 1.0 / 16, "INT4": 2.0 + 0.5 + 2.0 / 128}
-
-
 def _act_decode(dq, out, fmt, T, n):
     """Decoded activation d * q (binary32) from dq_act_quant's outputs, with the library's
     own codecs on the device."""
@@ -767,6 +1118,9 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.cpu_plan:
+            if rank == 0:
+                run_cpu_plan(args)
         elif args.gemm:
             run_gemm(args, world, rank, local)
         elif args.act:
