@@ -16,9 +16,11 @@
 // once per warp. A block of B channels spans B/16 lanes, which combine their absolute maxima
 // with xor shuffles; the block scale (two correctly rounded divisions and a reciprocal) is
 // computed once per 16 elements. The quantization pass loads the next row's chunk before it
-// works on the current one. NVFP4 needs the global amax of x~ first (a separate pass that
-// keeps AMAX_UNROLL rows of chunks in flight per lane; X is usually still in L2 for the
-// second read).
+// works on the current one. NVFP4 needs the global amax of x~ first: a separate pass that
+// keeps AMAX_UNROLL rows of chunks in flight per lane and writes one maximum per CTA (no
+// atomics, nothing to clear beforehand); the quantization pass is launched as its
+// programmatic dependent, so its launch overlaps the pre-pass, and it reduces those maxima
+// itself once the pre-pass has completed (X is usually still in L2 for its second read).
 #include <algorithm>
 
 #include "dq_device.cuh"
@@ -30,7 +32,6 @@ namespace {
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int ACT_WARPS = 8;
 constexpr int CHUNK = 16;                 // channels per lane and round
-constexpr int AMAX_UNROLL = 4;            // chunks per lane in flight in the amax pass
 constexpr int STRIP = CHUNK * 32;         // channels of one warp's strip
 
 // 16 channels as raw words (bf16: 8 words; fp32: 16 words)
@@ -39,27 +40,44 @@ struct Chunk {
   uint32_t u[F32IN ? 16 : 8];
 };
 
-template <bool F32IN>
-__device__ __forceinline__ void load_chunk(const void* X, int64_t row, int64_t ldx,
-                                           int64_t col, Chunk<F32IN>& d) {
-  if constexpr (F32IN) {
-    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(X) +
-                                                    row * ldx + col);
+// A lane's copy-ahead ring in shared memory: its chunks of the next RD rows are in flight as
+// asynchronous copies (no registers held) while it works on the current row. Every lane
+// copies and reads only its own slots, so no lane waits on another. Chunk h of lane l sits
+// at l*CB + (h ^ swizzle(l)), which spreads a quarter warp's 16-byte reads over all banks.
+template <bool F32IN, int RD>
+struct LaneRing {
+  static constexpr int CB = F32IN ? 4 : 2;          // 16-byte chunks per lane and row
+  uint4* base;                                      // this warp's [RD][32 * CB] slots
+  int lane, sw;
+  __device__ __forceinline__ LaneRing(uint4* warp_base, int l)
+      : base(warp_base), lane(l), sw(CB == 2 ? ((l >> 2) & 1) : ((l >> 1) & 3)) {}
+  // row `row` (when `in`; zeros otherwise) into slot `slot`; one commit group per call
+  __device__ __forceinline__ void issue(const void* X, int64_t row, int64_t ldx, int64_t col,
+                                        bool in, int slot) const {
+    if (in) {
+      const char* src = reinterpret_cast<const char*>(X) + (row * ldx + col) * (F32IN ? 4 : 2);
+      const uint32_t dst = static_cast<uint32_t>(
+          __cvta_generic_to_shared(base + (size_t)slot * 32 * CB + lane * CB));
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const uint4 v = __ldg(p + h);
-      d.u[4 * h] = v.x; d.u[4 * h + 1] = v.y; d.u[4 * h + 2] = v.z; d.u[4 * h + 3] = v.w;
+      for (int h = 0; h < CB; ++h)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                     :: "r"(dst + 16u * (uint32_t)(h ^ sw)), "l"(src + 16 * h) : "memory");
     }
-  } else {
-    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(X) +
-                                                    row * ldx + col);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  // the chunk of the oldest pending row, in slot `slot`, once its copy has landed
+  __device__ __forceinline__ void read(int slot, Chunk<F32IN>& d) const {
+    asm volatile("cp.async.wait_group %0;" :: "n"(RD - 1) : "memory");
+    const uint4* q = base + (size_t)slot * 32 * CB + lane * CB;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint4 v = __ldg(p + h);
+    for (int h = 0; h < CB; ++h) {
+      const uint4 v = q[h ^ sw];
       d.u[4 * h] = v.x; d.u[4 * h + 1] = v.y; d.u[4 * h + 2] = v.z; d.u[4 * h + 3] = v.w;
     }
   }
-}
+};
+constexpr int AMAX_RING = 5;              // rows in flight per lane, amax pass
+constexpr int QUANT_RING = 5;             // rows in flight per lane, quantization pass
 
 template <bool F32IN>
 __device__ __forceinline__ void zero_chunk(Chunk<F32IN>& d) {
@@ -123,6 +141,8 @@ __device__ __forceinline__ WarpWork warp_work(const ActLaunch& A, int64_t wps, i
 
 template <bool F32IN>
 __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int strips) {
+  // the quantization pass may start launching now; it waits for this grid's completion
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const WarpWork ww = warp_work(A, wps, strips);
   const int64_t col = ww.col, row0 = ww.row0, row1 = ww.row1;
@@ -130,26 +150,26 @@ __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int 
   float2 cv[8];
   load_c16(A.c, col, valid, cv);
   float a = 0.0f;
-  // AMAX_UNROLL rows per step, all their loads issued before any use (no stores here)
-  for (int64_t r0 = row0; r0 < row1; r0 += AMAX_UNROLL) {
-    Chunk<F32IN> d[AMAX_UNROLL];
+  constexpr int RD = F32IN ? AMAX_RING / 2 : AMAX_RING;
+  __shared__ __align__(16) uint4 ring_mem[ACT_WARPS][RD * 32 * LaneRing<F32IN, RD>::CB];
+  const LaneRing<F32IN, RD> ring(ring_mem[threadIdx.x / 32], lane);
 #pragma unroll
-    for (int u = 0; u < AMAX_UNROLL; ++u) {
-      if (valid && r0 + u < row1) load_chunk<F32IN>(A.X, r0 + u, A.ldx, col, d[u]);
-      else zero_chunk<F32IN>(d[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < AMAX_UNROLL; ++u) {
-      float2 x[8];
-      rescale_chunk<F32IN>(d[u], cv, x);
-      a = max_nan(a, absmax16(x));
-    }
+  for (int j = 0; j < RD; ++j) ring.issue(A.X, row0 + j, A.ldx, col, valid && row0 + j < row1, j);
+  int slot = 0;
+  for (int64_t row = row0; row < row1; ++row) {
+    Chunk<F32IN> d;
+    ring.read(slot, d);
+    if (!valid) zero_chunk<F32IN>(d);       // a lane past the last channel copied nothing
+    float2 x[8];
+    rescale_chunk<F32IN>(d, cv, x);        // the chunk is in registers: its slot is free
+    ring.issue(A.X, row + RD, A.ldx, col, valid && row + RD < row1, slot);
+    a = max_nan(a, absmax16(x));
+    slot = (slot + 1 == RD) ? 0 : slot + 1;
   }
   const bool bad = !isfinite(a);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL, a, off));
-  // one atomic per CTA: the maxima of its warps meet in shared memory first (every warp of
-  // the launch updating one word serialises at its L2 slice)
+  // one maximum per CTA, written to its own slot (the quantization pass reduces them)
   __shared__ float wmax[ACT_WARPS];
   if (lane == 0) wmax[threadIdx.x / 32] = a;
   __syncthreads();
@@ -157,7 +177,7 @@ __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int 
     float m = 0.0f;
 #pragma unroll
     for (int w = 0; w < ACT_WARPS; ++w) m = fmaxf(m, wmax[w]);
-    if (m > 0.0f) atomicMax(A.amax_bits, __float_as_uint(m));
+    A.partials[blockIdx.x] = __float_as_uint(m);
   }
   if (bad) atomicOr(A.err_word, ERRBIT_NONFINITE);
 }
@@ -178,9 +198,48 @@ __device__ __forceinline__ uint32_t e2m1x8_encode(const float2 (&y)[4]) {
   return out;
 }
 
+// The quantized codes of one 16-channel chunk on an integer grid (INT4 -7..7, INT8
+// -127..127): y = fl32(x * inv) clamped to [-Q, Q], then rounded to the nearest integer
+// (ties to even) by adding 1.5 * 2^23, whose last byte is then the integer's two's
+// complement. INT4: eight nibbles per word (value k in nibble k); INT8: four bytes per word.
+template <int ELEM>
+__device__ __forceinline__ void int_codes(const float2 (&x)[8], float2 iv, uint32_t (&w)[4]) {
+  constexpr float Q = elem_qmax<ELEM>();
+  const float2 magic = make_float2(12582912.0f, 12582912.0f), one = make_float2(1.0f, 1.0f);
+  uint32_t b[16];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    float2 y = mul2(x[p], iv);
+    y.x = fminf(fmaxf(y.x, -Q), Q);
+    y.y = fminf(fmaxf(y.y, -Q), Q);
+    const float2 z = fma2(y, one, magic);
+    b[2 * p] = __float_as_uint(z.x);
+    b[2 * p + 1] = __float_as_uint(z.y);
+  }
+  if constexpr (ELEM == ELEM_INT8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      w[k] = __byte_perm(__byte_perm(b[4 * k], b[4 * k + 1], 0x0040),
+                         __byte_perm(b[4 * k + 2], b[4 * k + 3], 0x0040), 0x5410);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint32_t by[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        // byte j: nibble of value 2j in the low half, of value 2j+1 in the high half
+        const uint32_t lo = b[8 * k + 2 * j], hi = b[8 * k + 2 * j + 1] << 4;
+        by[j] = (lo & 0x0Fu) | (hi & 0xF0u);
+      }
+      w[k] = __byte_perm(__byte_perm(by[0], by[1], 0x0040), __byte_perm(by[2], by[3], 0x0040),
+                         0x5410);
+    }
+  }
+}
+
 template <int ELEM, int SCALE, int B, bool F32IN>
 __global__ void __launch_bounds__(ACT_WARPS * 32, 3)
-act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
+act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips, const int nparts) {
   constexpr int LB = B / CHUNK;                   // lanes per block
   constexpr float QMAX = elem_qmax<ELEM>();
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
@@ -193,7 +252,20 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
   // NVFP4: every E4M3 code's decoded scale fl32(s_t * e) and its reciprocal, per CTA
   __shared__ float2 tbl[SCALE == SCALE_E4M3 ? 128 : 1];
   if constexpr (SCALE == SCALE_E4M3) {
-    s_t = nvfp4_tensor_scale(__uint_as_float(*A.amax_bits));
+    // the pre-pass (this grid's programmatic predecessor) has completed and its maxima are
+    // visible after the wait; every CTA reduces them (a few KB from L2)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ uint32_t pmax[ACT_WARPS];
+    uint32_t mx = 0u;
+    for (int i = threadIdx.x; i < nparts; i += blockDim.x) mx = max(mx, A.partials[i]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, off));
+    if ((threadIdx.x & 31) == 0) pmax[threadIdx.x / 32] = mx;
+    __syncthreads();
+    mx = 0u;
+#pragma unroll
+    for (int w = 0; w < ACT_WARPS; ++w) mx = max(mx, pmax[w]);
+    s_t = nvfp4_tensor_scale(__uint_as_float(mx));
     if (blockIdx.x == 0 && threadIdx.x == 0 && A.tensor_scale != nullptr) *A.tensor_scale = s_t;
     if (threadIdx.x < 128) {
       const uint32_t code = (threadIdx.x == 0 || threadIdx.x == 127) ? 1u : threadIdx.x;
@@ -209,15 +281,20 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
   float2 cv[8];
   load_c16(A.c, col, valid, cv);
   bool bad = false;
-  Chunk<F32IN> nxt;
-  if (valid && row0 < row1) load_chunk<F32IN>(A.X, row0, A.ldx, col, nxt);
-  else zero_chunk<F32IN>(nxt);
+  constexpr int RD = F32IN ? QUANT_RING / 2 : QUANT_RING;
+  __shared__ __align__(16) uint4 ring_mem[ACT_WARPS][RD * 32 * LaneRing<F32IN, RD>::CB];
+  const LaneRing<F32IN, RD> ring(ring_mem[threadIdx.x / 32], lane);
+#pragma unroll
+  for (int j = 0; j < RD; ++j) ring.issue(A.X, row0 + j, A.ldx, col, valid && row0 + j < row1, j);
+  int slot = 0;
   for (int64_t row = row0; row < row1; ++row) {
-    const Chunk<F32IN> cur = nxt;
-    // the next row's chunk is in flight while this one is quantized
-    if (valid && row + 1 < row1) load_chunk<F32IN>(A.X, row + 1, A.ldx, col, nxt);
+    Chunk<F32IN> cur;
+    ring.read(slot, cur);
+    if (!valid) zero_chunk<F32IN>(cur);     // a lane past the last channel copied nothing
     float2 x[8];
-    rescale_chunk<F32IN>(cur, cv, x);
+    rescale_chunk<F32IN>(cur, cv, x);      // the chunk is in registers: its slot is free
+    ring.issue(A.X, row + RD, A.ldx, col, valid && row + RD < row1, slot);
+    slot = (slot + 1 == RD) ? 0 : slot + 1;
     float a = absmax16(x);
     bad |= !isfinite(a);
 #pragma unroll
@@ -225,7 +302,7 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
     uint32_t code = 0;
     float inv = 0.0f;
     if (a > 0.0f) {
-      const ScaleVal sv = project_scale<SCALE>(__fdiv_rn(a, QMAX), s_t, tbl);
+      const ScaleVal sv = project_scale<SCALE>(div_qmax<(int)QMAX>(a), s_t, tbl);
       code = sv.code;
       inv = sv.ir;
     }
@@ -241,13 +318,7 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips) {
         w[h] = e2m1x8_encode(y);
       }
     } else {
-#pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        float2 q;
-        const uint32_t cb = quant2<ELEM>(mul2(x[p], iv), q);
-        if constexpr (BYTE_CODES) w[p >> 1] |= (cb & 0xFFFFu) << (16 * (p & 1));
-        else w[p >> 2] |= (cb & 0xFFu) << (8 * (p & 3));
-      }
+      int_codes<ELEM>(x, iv, w);
     }
     if (valid) {
       if (a == 0.0f) w[0] = w[1] = w[2] = w[3] = 0u;   // all-zero block: code 0 (also -0)
@@ -305,27 +376,55 @@ int64_t resident_warps() {
   return warps;
 }
 
-// launch over (strips x wps) warps: at most the resident warps, at least one row each
+// (strips x wps) warps: at most the resident warps (and cap_ctas CTAs), at least one row each
+struct RowGrid {
+  int strips;
+  int64_t wps, ctas;
+};
 template <auto KERNEL>
-cudaError_t launch_rows(const ActLaunch& A, cudaStream_t s) {
-  const int strips = (int)((A.n + STRIP - 1) / STRIP);
-  const int64_t wps = std::max<int64_t>(1, std::min<int64_t>(resident_warps<KERNEL>() / strips,
-                                                             A.tokens));
-  const int64_t ctas = (wps * strips + ACT_WARPS - 1) / ACT_WARPS;
-  KERNEL<<<(unsigned)ctas, ACT_WARPS * 32, 0, s>>>(A, wps, strips);
-  count_launches(1);
-  return cudaGetLastError();
+RowGrid row_grid(const ActLaunch& A, int64_t cap_ctas) {
+  RowGrid g;
+  g.strips = (int)((A.n + STRIP - 1) / STRIP);
+  const int64_t warps = std::min<int64_t>(resident_warps<KERNEL>(), cap_ctas * ACT_WARPS);
+  g.wps = std::max<int64_t>(1, std::min<int64_t>(warps / g.strips, A.tokens));
+  g.ctas = (g.wps * g.strips + ACT_WARPS - 1) / ACT_WARPS;
+  return g;
+}
+
+template <int ELEM, int SCALE, int B, bool F32IN>
+cudaError_t launch_fmt_dt(const ActLaunch& A, cudaStream_t s) {
+  constexpr auto QK = act_quant_kernel<ELEM, SCALE, B, F32IN>;
+  const RowGrid gq = row_grid<QK>(A, INT64_MAX / ACT_WARPS);
+  if constexpr (SCALE != SCALE_E4M3) {
+    QK<<<(unsigned)gq.ctas, ACT_WARPS * 32, 0, s>>>(A, gq.wps, gq.strips, 0);
+    count_launches(1);
+    return cudaGetLastError();
+  } else {
+    constexpr auto AK = act_amax_kernel<F32IN>;
+    const RowGrid ga = row_grid<AK>(A, ACT_MAX_PARTS);
+    AK<<<(unsigned)ga.ctas, ACT_WARPS * 32, 0, s>>>(A, ga.wps, ga.strips);
+    count_launches(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)gq.ctas);
+    cfg.blockDim = dim3(ACT_WARPS * 32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, QK, A, gq.wps, gq.strips, (int)ga.ctas);
+    count_launches(1);
+    return e;
+  }
 }
 
 template <int ELEM, int SCALE, int B>
 cudaError_t launch_fmt(const ActLaunch& A, int esize, cudaStream_t s) {
-  if (SCALE == SCALE_E4M3) {
-    const cudaError_t e = (esize == 4) ? launch_rows<act_amax_kernel<true>>(A, s)
-                                       : launch_rows<act_amax_kernel<false>>(A, s);
-    if (e != cudaSuccess) return e;
-  }
-  return (esize == 4) ? launch_rows<act_quant_kernel<ELEM, SCALE, B, true>>(A, s)
-                      : launch_rows<act_quant_kernel<ELEM, SCALE, B, false>>(A, s);
+  return (esize == 4) ? launch_fmt_dt<ELEM, SCALE, B, true>(A, s)
+                      : launch_fmt_dt<ELEM, SCALE, B, false>(A, s);
 }
 
 }  // namespace

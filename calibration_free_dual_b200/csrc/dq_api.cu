@@ -353,7 +353,8 @@ dq_status dq_w4a4_gemm(const uint8_t* x_packed, const uint8_t* x_scales,
 
 size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt) {
   if (tokens < 0 || n <= 0 || check_format(fmt) != DQ_OK) return 0;
-  return 256;
+  // NVFP4: one maximum per CTA of the amax pre-pass
+  return fmt.kind == DQ_NVFP4 ? (size_t)4 * dq::ACT_MAX_PARTS : 256;
 }
 
 dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, int64_t ldx,
@@ -388,16 +389,14 @@ dq_status dq_act_quant(const void* X, int32_t dtype, int64_t tokens, int64_t n, 
   A.x_packed = x_packed;
   A.scales = scales;
   A.tensor_scale = tensor_scale;
-  A.amax_bits = static_cast<unsigned*>(workspace);
+  A.partials = static_cast<unsigned*>(workspace);
   A.err_word = errp;
-  if (fmt.kind == DQ_NVFP4) {
-    if ((st = from_cuda(cudaMemsetAsync(workspace, 0, 4, s))) != DQ_OK) return st;
-  }
   return from_cuda(dq::launch_act(A, fmt.kind, fmt.group, esize, s));
 }
 
-// W4A4 linear layer: workspace = [amax word, activation tensor scale | activation codes |
-// activation scale factors in the tensor core's layout | weight scale factors re-laid]
+// W4A4 linear layer: workspace = [activation tensor scale | per-CTA maxima of the amax
+// pre-pass | activation codes | activation scale factors in the tensor core's layout |
+// weight scale factors re-laid]
 namespace {
 struct LinearWs {
   size_t codes, sfa, sfb, total;
@@ -405,7 +404,7 @@ struct LinearWs {
 LinearWs linear_ws(int64_t T, int64_t N, int64_t K) {
   LinearWs l;
   const int64_t tpad = (T + 127) / 128 * 128;
-  l.codes = 256;
+  l.codes = 256 + (size_t)4 * dq::ACT_MAX_PARTS;
   l.sfa = dq::align_up(l.codes + (size_t)T * (size_t)(K / 2), 256);
   l.sfb = dq::align_up(l.sfa + (size_t)tpad * (size_t)(K / 16), 256);
   l.total = l.sfb + dq::gemm_workspace_bytes(T, N, K, true);
@@ -448,8 +447,7 @@ dq_status dq_w4a4_linear(const void* X, int32_t dtype, int64_t T, int64_t K, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int64_t kq = K / 64;
-  // the amax word, and the scale factors of the rows past T in the last 128-row block
-  if ((st = from_cuda(cudaMemsetAsync(ws, 0, 4, s))) != DQ_OK) return st;
+  // the scale factors of the rows past T in the last 128-row block
   if (T % 128 != 0 &&
       (st = from_cuda(cudaMemsetAsync(ws + l.sfa + (T / 128) * kq * 512, 0, (size_t)kq * 512, s))) != DQ_OK)
     return st;
@@ -462,15 +460,15 @@ dq_status dq_w4a4_linear(const void* X, int32_t dtype, int64_t T, int64_t K, int
   act.c = c;
   act.x_packed = ws + l.codes;
   act.scales = ws + l.sfa;
-  act.tensor_scale = reinterpret_cast<float*>(ws + 4);
-  act.amax_bits = reinterpret_cast<unsigned*>(ws);
+  act.tensor_scale = reinterpret_cast<float*>(ws);
+  act.partials = reinterpret_cast<unsigned*>(ws + 256);
   act.err_word = errp;
   act.sf_tc = 1;
   if ((st = from_cuda(dq::launch_act(act, fmt.kind, fmt.group, esize, s))) != DQ_OK) return st;
   dq::GemmArgs A = {};
   A.xq = ws + l.codes;
   A.xs = nullptr;
-  A.xst = reinterpret_cast<const float*>(ws + 4);
+  A.xst = reinterpret_cast<const float*>(ws);
   A.wq = w_packed;
   A.ws = w_scales;
   A.wst = w_tensor_scale;

@@ -112,6 +112,9 @@ cudaError_t launch_finalize(double* const* mse, double* const* ws_err, double* c
                             double* const* qchange, double* const* ws_qch, const int* tiles,
                             int count, int T, cudaStream_t s);
 
+// NVFP4 activation pre-pass: at most this many CTAs, each writing its own maximum
+constexpr int ACT_MAX_PARTS = 4096;
+
 struct ActLaunch {
   const void* X;
   int64_t tokens, n, ldx;
@@ -119,7 +122,7 @@ struct ActLaunch {
   uint8_t* x_packed;
   void* scales;
   float* tensor_scale;
-  unsigned* amax_bits;
+  unsigned* partials;  // NVFP4: [ACT_MAX_PARTS] per-CTA amax of the pre-pass (float bits)
   unsigned* err_word;
   int sf_tc;          // NVFP4: scales in the tensor core's layout (see dq_gemm.h), else [tokens, n/16]
 };

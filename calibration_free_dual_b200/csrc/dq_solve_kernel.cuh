@@ -395,7 +395,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         if (M.r0 != nullptr) {
           v = (row < m) ? M.r0[(int64_t)row * nb + col0 / B + bl] : 1.0f;
         } else {
-          v = (a > 0.0f) ? __fdiv_rn(a, QMAX) : 1.0f;
+          v = (a > 0.0f) ? div_qmax<(int)QMAX>(a) : 1.0f;
         }
         sc = project_scale<SCALE>(v, s_t, tbl);
         old_code = sc.code;

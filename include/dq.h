@@ -181,7 +181,9 @@ DQ_API dq_status dq_solve_noalloc(const void* W, int32_t dtype, int64_t m, int64
 /* Largest m the solver handles for a given n, format and dtype (0 if the format is bad). */
 DQ_API int64_t dq_solve_max_rows(int64_t n, dq_format fmt, int32_t dtype);
 
-/* Workspace (device bytes) needed by dq_act_quant. */
+/* Workspace (device bytes) needed by dq_act_quant: for NVFP4, one slot per CTA of the
+ * amax pre-pass (16 KB; every call writes all the slots it reads, nothing needs clearing),
+ * otherwise 256 bytes. */
 DQ_API size_t dq_act_quant_workspace_bytes(int64_t tokens, int64_t n, dq_format fmt);
 
 /* Activation rescale + block quantization (DualQuant Abstract: the column scales are

@@ -129,9 +129,10 @@ def test_act_quant_offset_codes_and_strided_x(dq, fmt_name):
     sdt = torch.int16 if fmt.scale == "bf16" else torch.uint8
     scales = torch.empty((T, n // fmt.block), dtype=sdt, device="cuda")
     ts = torch.empty((1,), dtype=torch.float32, device="cuda")
-    ws = torch.empty((256,), dtype=torch.uint8, device="cuda")
-    cd = torch.from_numpy(c).cuda()
     lib = _lib.get()
+    ws = torch.empty((lib.dq_act_quant_workspace_bytes(T, n, f),), dtype=torch.uint8,
+                     device="cuda")
+    cd = torch.from_numpy(c).cuda()
     st = lib.dq_act_quant(ctypes.c_void_p(X.data_ptr()), _lib.DQ_BF16, T, n, ld,
                           ctypes.c_void_p(cd.data_ptr()), f, ctypes.c_void_p(base),
                           ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(ts.data_ptr()),
