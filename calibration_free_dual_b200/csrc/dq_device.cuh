@@ -174,10 +174,42 @@ __device__ __forceinline__ ScaleVal scale_decode(uint32_t code, const float2* tb
   return s;
 }
 
-// Nearest admissible scale to v (binary32): bf16 RNE clamped to [2^-126, max]; E8M0 nearest
-// power of two; E4M3: e = RNE(fl32(v / s_t)) raised to 2^-9 if 0, scale fl32(s_t * e).
+// A bf16 block scale from its code with 1/r from a table of the 128 mantissa reciprocals
+// rtab[f] = fl32(1 / (1 + f/128)): for a normal code with exponent field E <= 252, fl32(1/r)
+// is rtab[f] * 2^(127 - E) exactly (a power-of-two scaling that stays in the normal range),
+// formed by adding to the exponent bits; the two largest binades (a subnormal reciprocal)
+// take the correctly rounded reciprocal.
+__device__ __forceinline__ ScaleVal bf16_scale_decode_tab(uint32_t code, const float* rtab) {
+  ScaleVal s;
+  s.code = code;
+  s.r = __uint_as_float(code << 16);
+  const uint32_t E = (code >> 7) & 0xFFu;
+  s.ir = (E <= 252u) ? __uint_as_float(__float_as_uint(rtab[code & 0x7Fu]) + ((127u - E) << 23))
+                     : __frcp_rn(s.r);
+  return s;
+}
+
+// fl32(num / den) for binary64 num >= 0, den > 0 (normal), by a reciprocal: the hardware's
+// approximate binary64 reciprocal refined by two Newton-Raphson steps y <- y + y(1 - den y)
+// (each squares the relative error), so that num * y is within a few binary64 ulps of the
+// quotient before its rounding to binary32. It can differ from fl32 of the correctly rounded
+// binary64 quotient only within a few binary64 ulps of a binary32 midpoint, far inside the
+// rounding of the binary64 sums num and den themselves.
+__device__ __forceinline__ float div64_to_f32(double num, double den) {
+  double y;
+  asm("rcp.approx.ftz.f64 %0, %1;" : "=d"(y) : "d"(den));
+  double e = fma(-den, y, 1.0);
+  y = fma(y, e, y);
+  e = fma(-den, y, 1.0);
+  y = fma(y, e, y);
+  return __double2float_rn(num * y);
+}
+
+// Nearest admissible scale to v (binary32), as a code: bf16 RNE clamped to [2^-126, max];
+// E8M0 nearest power of two; E4M3: e = RNE(fl32(v / s_t)) raised to 2^-9 if 0 (the scale is
+// then fl32(s_t * e)).
 template <int SCALE>
-__device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const float2* tbl) {
+__device__ __forceinline__ uint32_t project_code(float v, float s_t) {
   uint32_t code;
   if constexpr (SCALE == SCALE_BF16) {
     code = (v > 0.0f) ? bf16_rn_bits(v) : 0x0080u;
@@ -188,7 +220,13 @@ __device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const floa
     float u = (v > 0.0f) ? __fdiv_rn(v, s_t) : 0.0f;
     code = max(e4m3_encode(u), 1u);
   }
-  return scale_decode<SCALE>(code, tbl);
+  return code;
+}
+
+// The same projection, decoded.
+template <int SCALE>
+__device__ __forceinline__ ScaleVal project_scale(float v, float s_t, const float2* tbl) {
+  return scale_decode<SCALE>(project_code<SCALE>(v, s_t), tbl);
 }
 
 // Projection of the least-squares scale num/den inside a BCD iteration. The quotient is a

@@ -214,8 +214,13 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     }
   }
 
-  // ---- tensor scale (NVFP4) and the code -> (r, 1/r) table
+  // ---- tensor scale (NVFP4) and the code -> (r, 1/r) table; bf16 scales: the table of
+  // mantissa reciprocals
   float s_t = 1.0f;
+  const float* rtab = reinterpret_cast<const float*>(tbl);
+  if constexpr (SCALE == SCALE_BF16) {
+    if (tid < 128) reinterpret_cast<float*>(tbl)[tid] = __frcp_rn(1.0f + (float)tid * 0.0078125f);
+  }
   if constexpr (SCALE == SCALE_E4M3) {
     s_t = nvfp4_tensor_scale(__uint_as_float(*M.amax_bits));
     if (tid < 128) {
@@ -317,6 +322,12 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
 
   double wsq_tile = 0.0;    // ||W||^2 of the tile (thread 0)
 
+  // code -> scale: bf16 scales with the reciprocal table, the others as before
+  auto dec = [&](uint32_t code) -> ScaleVal {
+    if constexpr (SCALE == SCALE_BF16) return bf16_scale_decode_tab(code, rtab);
+    else return scale_decode<SCALE>(code, tbl);
+  };
+
   // One pass over all rows of the tile. INIT: iteration 0 (scales from absmax or r0,
   // c = c0); otherwise one BCD iteration (Q-step, r-step + projection, c-step). EMIT: the
   // returned state is written.
@@ -343,7 +354,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     Raw<ESZ> buf;
     fetch(0, buf);
     ScaleVal scn;
-    if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(0), tbl);
+    if constexpr (!INIT) scn = dec(code_at(0));
     // one row step; NEXT: which source the next row comes from (0: none, this is the last
     // row; 1: shared memory; 2: L2, or zeros past the last row; 3: tested per row; 4: L2, a
     // sweep with every row below m, 256-bit loads). With SPLIT_ROWS the source is fixed per
@@ -378,10 +389,10 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       if constexpr (NEXT == 3) {
         if (k + 1 < RPT) {
           fetch(k + 1, buf);
-          if constexpr (!INIT) scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+          if constexpr (!INIT) scn = dec(code_at(k + 1));
         }
       } else if constexpr (!INIT && NEXT != 0) {
-        scn = scale_decode<SCALE>(code_at(k + 1), tbl);
+        scn = dec(code_at(k + 1));
       }
       if constexpr (INIT) {
         // NaN-propagating maximum: a is non-finite exactly when one of the piece's values is
@@ -397,7 +408,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
         } else {
           v = (a > 0.0f) ? div_qmax<(int)QMAX>(a) : 1.0f;
         }
-        sc = project_scale<SCALE>(v, s_t, tbl);
+        sc = dec(project_code<SCALE>(v, s_t));
         old_code = sc.code;
       }
 
@@ -424,7 +435,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       if constexpr (EXT && !INIT) {
         if (qch && t >= 2) {
           // q of the previous iteration, from its (r, c)
-          const ScaleVal sp = scale_decode<SCALE>(pcode_at(k), tbl);
+          const ScaleVal sp = dec(pcode_at(k));
           const float2 irp = make_float2(sp.ir, sp.ir);
           const float4* pv = reinterpret_cast<const float4*>(picvec + s * 16);
 #pragma unroll
@@ -463,7 +474,7 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
             num += __shfl_xor_sync(FULL, num, off);
             den += __shfl_xor_sync(FULL, den, off);
           }
-          if (den > 0.0) sc = project_scale<SCALE>(__double2float_rn(num / den), s_t, tbl);
+          if (den > 0.0) sc = dec(project_code<SCALE>(div64_to_f32(num, den), s_t));
         } else {
           float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
 #pragma unroll
