@@ -563,7 +563,10 @@ def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dic
     NVFP4 and INT4 g=128: device time per call with L2 flushed before it, the HBM fraction
     on the algorithmic bytes, and the SQNR of the decoded activation with and without c."""
     T, n = X.shape
-    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)    # 2x the 126 MB L2
+    # 2x the 126 MB L2: one buffer written, then one read, so that L2 holds none of X and no
+    # dirty lines whose write-back would land inside the timed call
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    flush_r = torch.ones((64 << 20,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     res = {}
     launches = 0
@@ -578,6 +581,7 @@ def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dic
         l0 = lib.dq_kernel_launches()
         for e0, e1 in evs:
             flush.fill_(1)                     # L2 holds none of X when the call starts
+            flush_r.amax()
             # a GPU-side wait of ~1 ms lets the host enqueue the whole call before e0 is
             # reached, so the events see the call's device time alone
             torch.cuda._sleep(2_000_000)
@@ -597,10 +601,10 @@ def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dic
                     "roofline": hbm_roofline(ACT_BYTES_PER_ELEM[fmt] * T * n, ms, peaks,
                                              peak_src, bytes_per_elem=ACT_BYTES_PER_ELEM[fmt],
                                              traffic=None)}
-    del flush
+    del flush, flush_r
     return {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) times the "
-                        "step's block-0 k_proj c; L2 flushed (256 MB written) before every "
-                        "call; device time of the call (its kernels), enqueued through the C "
+                        "step's block-0 k_proj c; L2 flushed before every call (256 MB "
+                        "written, then 256 MB read, so no dirty lines are left); device time of the call (its kernels), enqueued through the C "
                         "ABI with preallocated outputs behind a 1 ms GPU-side wait",
             "formats": res, "gpu_launches": int(launches)}
 
@@ -1076,7 +1080,10 @@ def run_act(args, world, rank, local):
     c = dq.solve(Wk, "MXFP4", wl.ACT_KPROJ.iters)["c"]
     X = wl.act_device(seed=wl.ACT_SEED + rank, device=dev)
     T, n = X.shape
-    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)    # 2x the 126 MB L2
+    # 2x the 126 MB L2: one buffer written, then one read, so that L2 holds none of X and no
+    # dirty lines whose write-back would land inside the timed call
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    flush_r = torch.ones((64 << 20,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = _lib.get()
     peaks, peak_src = _peaks()
@@ -1096,6 +1103,7 @@ def run_act(args, world, rank, local):
         l0 = lib.dq_kernel_launches()
         for e0, e1 in evs:
             flush.fill_(1)                     # L2 holds none of X when the call starts
+            flush_r.amax()
             # a GPU-side wait of ~1 ms lets the host enqueue the whole call before e0 is
             # reached, so the events see the call's device time alone
             torch.cuda._sleep(2_000_000)
@@ -1130,7 +1138,8 @@ def run_act(args, world, rank, local):
             "config": {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) "
                                    "times a k_proj's c (1024 x 4096, MXFP4 solve), NVFP4 "
                                    "(amax pass + quantization pass); INT4 g=128 alongside",
-                       "l2": "flushed (256 MB written) before every timed call",
+                       "l2": "flushed before every timed call (256 MB written, then 256 MB "
+                             "read: no dirty lines left)",
                        "timed": "device time of each call (its kernels), enqueued through the C "
                                 "ABI with preallocated outputs behind a 1 ms GPU-side wait"},
             "roofline": dict(head["roofline"], kernel="act_amax_kernel + act_quant_kernel"),

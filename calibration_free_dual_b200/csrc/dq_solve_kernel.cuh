@@ -457,24 +457,54 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
       if (ITER && upd_r) {
         // r-step: least squares over the block, then projection
         if constexpr (SCALE == SCALE_BF16) {
-          // INT4's fine bf16 scale grid: block sums in binary64 keep projection decisions
-          // on the exact least-squares quotient
-          double num = 0.0, den = 0.0;
+          // The fine bf16 scale grid: the block sums in binary32 first. Every term is >= 0
+          // (a code has the sign of its weight), so the binary32 sums carry a relative error
+          // of at most 13 and 14 units of binary32 rounding (the longest chain of roundings:
+          // the product q c, 8 accumulations, the pair, 3 shuffle levels), and the correctly
+          // rounded quotient v at most 28, i.e. under 28 ulps of v. bf16 rounds at the
+          // binary32 patterns whose low 16 bits are 0x8000, so a v more than 128 ulps from one
+          // (and inside [2^-90, 2^126), where neither underflow nor the clamps play a part)
+          // rounds as the exact least-squares quotient does. Otherwise (about 0.4% of the
+          // blocks, and every empty block) the block sums are taken again in binary64.
+          float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
-            const double qcx = (double)q[p].x * (double)cc[p].x;
-            const double qcy = (double)q[p].y * (double)cc[p].y;
-            num = fma((double)w[p].x, qcx, num);
-            num = fma((double)w[p].y, qcy, num);
-            den = fma(qcx, qcx, den);
-            den = fma(qcy, qcy, den);
+            const float2 qc = mul2(q[p], cc[p]);
+            num2 = fma2(w[p], qc, num2);
+            den2 = fma2(qc, qc, den2);
           }
+          float num = num2.x + num2.y, den = den2.x + den2.y;
 #pragma unroll
           for (int off = 1; off < LPB; off <<= 1) {
             num += __shfl_xor_sync(FULL, num, off);
             den += __shfl_xor_sync(FULL, den, off);
           }
-          if (den > 0.0) sc = dec(project_code<SCALE>(div64_to_f32(num, den), s_t));
+          const float v = __fdiv_rn(num, den);
+          const uint32_t lo = __float_as_uint(v) & 0xFFFFu;
+          const bool sure = num >= 0x1p-90f && den >= 0x1p-90f && v >= 0x1p-90f &&
+                            v < 0x1p126f && (lo + 128u - 0x8000u) > 256u;
+          uint32_t code = project_code<SCALE>(v, s_t);
+          if (__any_sync(FULL, !sure)) {
+            double num64 = 0.0, den64 = 0.0;
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+              const double qcx = (double)q[p].x * (double)cc[p].x;
+              const double qcy = (double)q[p].y * (double)cc[p].y;
+              num64 = fma((double)w[p].x, qcx, num64);
+              num64 = fma((double)w[p].y, qcy, num64);
+              den64 = fma(qcx, qcx, den64);
+              den64 = fma(qcy, qcy, den64);
+            }
+#pragma unroll
+            for (int off = 1; off < LPB; off <<= 1) {
+              num64 += __shfl_xor_sync(FULL, num64, off);
+              den64 += __shfl_xor_sync(FULL, den64, off);
+            }
+            if (!sure)
+              code = (den64 > 0.0) ? project_code<SCALE>(div64_to_f32(num64, den64), s_t)
+                                   : sc.code;
+          }
+          sc = dec(code);
         } else {
           float2 num2 = make_float2(0.f, 0.f), den2 = make_float2(0.f, 0.f);
 #pragma unroll
