@@ -558,54 +558,90 @@ def act_call_prepared(dq, lib, X, fmt, c):
 
 
 
-def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dict:
-    """dq_act_quant alone on the activation workload (8192 x 4096 bf16) with column scales c,
-    NVFP4 and INT4 g=128: device time per call with L2 flushed before it, the HBM fraction
-    on the algorithmic bytes, and the SQNR of the decoded activation with and without c."""
-    T, n = X.shape
-    # 2x the 126 MB L2: one buffer written, then one read, so that L2 holds none of X and no
-    # dirty lines whose write-back would land inside the timed call
+ACT_ROTATE = 4          # distinct activation inputs cycled by the back-to-back timing
+
+
+def act_timings(dq, lib, X, c, fmt, dev, steps, warmup, world):
+    """Device time of dq_act_quant on X (through the C ABI, preallocated outputs), two ways:
+
+    - streamed: `steps` calls back to back between one pair of events, cycling over
+      ACT_ROTATE copies of X with their own outputs (together larger than the 126 MB L2, so
+      no call finds its input in L2), after an L2 flush; time per call = total / steps. This
+      is the throughput of a stream of calls, the figure the roofline divides.
+    - isolated: one call per event pair, L2 flushed before it (256 MB written, then 256 MB
+      read, so no dirty lines are left to write back inside the call) and a 1 ms GPU-side
+      wait so that the host has enqueued the call; this adds the launch and event latency
+      (about 6 us on an empty kernel) to every call.
+
+    Returns (streamed ms, isolated ms, outputs of one call, kernel launches counted)."""
     flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
     flush_r = torch.ones((64 << 20,), dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    Xs = [X] + [X.clone() for _ in range(ACT_ROTATE - 1)]
+    calls = [act_call_prepared(dq, lib, Xi, fmt, c) for Xi in Xs]
+    for _ in range(max(warmup, 1)):
+        for call in calls:
+            call(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    l0 = lib.dq_kernel_launches()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush.fill_(1)
+    flush_r.amax()
+    torch.cuda._sleep(2_000_000)
+    e0.record(stream)
+    for i in range(steps):
+        out = calls[i % ACT_ROTATE](stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    streamed = e0.elapsed_time(e1) / steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        flush.fill_(1)
+        flush_r.amax()
+        torch.cuda._sleep(2_000_000)
+        a.record(stream)
+        calls[0](stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = lib.dq_kernel_launches() - l0
+    if dq.last_device_error() != 0:
+        raise RuntimeError("device error during the activation timing")
+    isolated = sum(a.elapsed_time(b) for a, b in evs) / steps
+    del flush, flush_r, Xs, calls
+    return reduce_max(streamed, world), reduce_max(isolated, world), out, launches
+
+
+def act_timing_text(steps: int) -> str:
+    return ("device time per call over %d calls back to back through the C ABI (preallocated "
+            "outputs), cycling over %d copies of X (268 MB, larger than L2); isolated: one "
+            "call behind an L2 flush (256 MB written, then read) and a 1 ms GPU-side wait"
+            % (steps, ACT_ROTATE))
+
+
+def act_record(dq, lib, X, c, dev, steps, warmup, world, peaks, peak_src) -> dict:
+    """dq_act_quant alone on the activation workload (8192 x 4096 bf16) with column scales c,
+    NVFP4 and INT4 g=128: device time per call (streamed and isolated, see act_timings), the
+    HBM fraction on the algorithmic bytes, and the SQNR of the decoded activation with and
+    without c."""
+    T, n = X.shape
     res = {}
     launches = 0
     for fmt in ("NVFP4", "INT4"):
-        call = act_call_prepared(dq, lib, X, fmt, c)
-        for _ in range(max(warmup, 1)):
-            call(stream)
-        torch.cuda.synchronize(dev)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        barrier(world)
-        l0 = lib.dq_kernel_launches()
-        for e0, e1 in evs:
-            flush.fill_(1)                     # L2 holds none of X when the call starts
-            flush_r.amax()
-            # a GPU-side wait of ~1 ms lets the host enqueue the whole call before e0 is
-            # reached, so the events see the call's device time alone
-            torch.cuda._sleep(2_000_000)
-            e0.record(stream)
-            out = call(stream)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        launches += lib.dq_kernel_launches() - l0
-        if dq.last_device_error() != 0:
-            raise RuntimeError("device error during the activation timing")
-        ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / steps, world)
+        ms, ms_iso, out, nl = act_timings(dq, lib, X, c, fmt, dev, steps, warmup, world)
+        launches += nl
         sq = {"with_c": _sqnr(X.float() * c, _act_decode(dq, out, fmt, T, n))}
         out0 = dq.act_quant(X, fmt, None)
         sq["without_c"] = _sqnr(X.float(), _act_decode(dq, out0, fmt, T, n))
-        res[fmt] = {"us_per_call": ms * 1e3, "elems_per_s": world * T * n / (ms * 1e-3),
-                    "sqnr_db": sq,
+        res[fmt] = {"us_per_call": ms * 1e3, "us_per_call_isolated": ms_iso * 1e3,
+                    "elems_per_s": world * T * n / (ms * 1e-3), "sqnr_db": sq,
                     "roofline": hbm_roofline(ACT_BYTES_PER_ELEM[fmt] * T * n, ms, peaks,
                                              peak_src, bytes_per_elem=ACT_BYTES_PER_ELEM[fmt],
                                              traffic=None)}
-    del flush, flush_r
     return {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) times the "
-                        "step's block-0 k_proj c; L2 flushed before every call (256 MB "
-                        "written, then 256 MB read, so no dirty lines are left); device time of the call (its kernels), enqueued through the C "
-                        "ABI with preallocated outputs behind a 1 ms GPU-side wait",
+                        "step's block-0 k_proj c",
+            "timing": act_timing_text(steps),
             "formats": res, "gpu_launches": int(launches)}
 
 
@@ -1079,71 +1115,29 @@ def run_act(args, world, rank, local):
     Wk = wl.weight_device(wl.ACT_KPROJ, 0, 1, device=dev, seed_offset=rank)
     c = dq.solve(Wk, "MXFP4", wl.ACT_KPROJ.iters)["c"]
     X = wl.act_device(seed=wl.ACT_SEED + rank, device=dev)
-    T, n = X.shape
-    # 2x the 126 MB L2: one buffer written, then one read, so that L2 holds none of X and no
-    # dirty lines whose write-back would land inside the timed call
-    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
-    flush_r = torch.ones((64 << 20,), dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream(dev)
     lib = _lib.get()
     peaks, peak_src = _peaks()
-    res = {}
-    launches = 0
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    for fmt in ("NVFP4", "INT4"):
-        call = act_call_prepared(dq, lib, X, fmt, c)
-        for _ in range(args.warmup):
-            call(stream)
-        torch.cuda.synchronize(dev)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        barrier(world)
-        l0 = lib.dq_kernel_launches()
-        for e0, e1 in evs:
-            flush.fill_(1)                     # L2 holds none of X when the call starts
-            flush_r.amax()
-            # a GPU-side wait of ~1 ms lets the host enqueue the whole call before e0 is
-            # reached, so the events see the call's device time alone
-            torch.cuda._sleep(2_000_000)
-            e0.record(stream)
-            out = call(stream)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        launches += lib.dq_kernel_launches() - l0
-        if dq.last_device_error() != 0:
-            raise RuntimeError("device error during the timed region")
-        ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / args.steps, world)
-        sq = {"with_c": _sqnr(X.float() * c, _act_decode(dq, out, fmt, T, n))}
-        out0 = dq.act_quant(X, fmt, None)
-        sq["without_c"] = _sqnr(X.float(), _act_decode(dq, out0, fmt, T, n))
-        gbs = ACT_BYTES_PER_ELEM[fmt] * T * n / (ms * 1e-3) / 1e9
-        res[fmt] = {"ms_per_call": ms, "elems_per_s": world * T * n / (ms * 1e-3),
-                    "sqnr_db": sq,
-                    "roofline": {"bound": "hbm", "achieved": gbs,
-                                 "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                                 "frac": gbs / float(peaks["hbm_gbs"]), "traffic": None,
-                                 "bytes_per_elem": ACT_BYTES_PER_ELEM[fmt],
-                                 "peak_source": peak_src}}
+    rec = act_record(dq, lib, X, c, dev, args.steps, args.warmup, world, peaks, peak_src)
     clk = clocks.stop()
     if rank == 0:
-        head = res["NVFP4"]
+        head = rec["formats"]["NVFP4"]
         line = {
             "metric": "activation rescale+quantize elements/s",
             "value": head["elems_per_s"], "unit": "elem/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_call"],
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["us_per_call"] / 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": {"workload": "activations 8192 x 4096 bf16 (N(0,1), 6 channels x50) "
                                    "times a k_proj's c (1024 x 4096, MXFP4 solve), NVFP4 "
                                    "(amax pass + quantization pass); INT4 g=128 alongside",
-                       "l2": "flushed before every timed call (256 MB written, then 256 MB "
-                             "read: no dirty lines left)",
-                       "timed": "device time of each call (its kernels), enqueued through the C "
-                                "ABI with preallocated outputs behind a 1 ms GPU-side wait"},
+                       "l2": "inputs larger than L2 (%d copies of X cycled); the isolated "
+                             "figure flushes L2 before each call" % ACT_ROTATE,
+                       "timed": rec["timing"]},
             "roofline": dict(head["roofline"], kernel="act_amax_kernel + act_quant_kernel"),
-            "formats": res, "gpu_launches": int(launches), "clocks": clk,
+            "formats": rec["formats"], "gpu_launches": rec["gpu_launches"], "clocks": clk,
         }
         print(json.dumps(line), flush=True)
 

@@ -8,19 +8,19 @@
 // data. With W_hat = diag(r) Q diag(c) the quantized GEMM consumes c * x, so the kernel
 // quantizes x~ = fl32(X * c).
 //
-// Layout of the work: the launch holds as many warps as the SMs keep resident; each warp owns
-// a strip of 512 channels and an equal share of the token rows (a contiguous range), each
-// lane a chunk of 16 consecutive channels of the strip (bf16: two 16-byte loads); a lane
-// keeps its 16 column scales in registers for all its rows and walks down the rows, so a
-// warp's loads, its 8-byte code stores and its scale stores are contiguous and c is read
-// once per warp. A block of B channels spans B/16 lanes, which combine their absolute maxima
-// with xor shuffles; the block scale (two correctly rounded divisions and a reciprocal) is
-// computed once per 16 elements. The quantization pass loads the next row's chunk before it
-// works on the current one. NVFP4 needs the global amax of x~ first: a separate pass that
-// keeps AMAX_UNROLL rows of chunks in flight per lane and writes one maximum per CTA (no
-// atomics, nothing to clear beforehand); the quantization pass is launched as its
-// programmatic dependent, so its launch overlaps the pre-pass, and it reduces those maxima
-// itself once the pre-pass has completed (X is usually still in L2 for its second read).
+// Layout of the work: each warp owns a strip of 512 channels and a contiguous range of token
+// rows (rows per warp set on the host so that the launch holds about as many warps as the SMs
+// keep resident); each lane owns a chunk of 16 consecutive channels of the strip, keeps its
+// 16 column scales in registers for all its rows and walks down the rows, so a warp's loads,
+// its 8-byte code stores and its scale stores are contiguous and c is read once per warp.
+// Rows arrive through a per-lane ring of asynchronous copies in shared memory (several rows
+// in flight, no registers held). A block of B channels spans B/16 lanes, which combine their
+// absolute maxima with xor shuffles; the block scale is computed once per 16 elements. NVFP4
+// needs the global amax of x~ first: a separate pass over the same rows that writes one
+// maximum per CTA (no atomics, nothing to clear beforehand); the quantization pass is launched
+// as its programmatic dependent, so its launch overlaps the pre-pass, and it reduces those
+// maxima itself once the pre-pass has completed (X is usually still in L2 for its second
+// read).
 #include <algorithm>
 
 #include "dq_device.cuh"
@@ -51,11 +51,9 @@ struct LaneRing {
   int lane, sw;
   __device__ __forceinline__ LaneRing(uint4* warp_base, int l)
       : base(warp_base), lane(l), sw(CB == 2 ? ((l >> 2) & 1) : ((l >> 1) & 3)) {}
-  // row `row` (when `in`; zeros otherwise) into slot `slot`; one commit group per call
-  __device__ __forceinline__ void issue(const void* X, int64_t row, int64_t ldx, int64_t col,
-                                        bool in, int slot) const {
+  // the lane's chunk at `src` (when `in`) into slot `slot`; one commit group per call
+  __device__ __forceinline__ void issue(const char* src, bool in, int slot) const {
     if (in) {
-      const char* src = reinterpret_cast<const char*>(X) + (row * ldx + col) * (F32IN ? 4 : 2);
       const uint32_t dst = static_cast<uint32_t>(
           __cvta_generic_to_shared(base + (size_t)slot * 32 * CB + lane * CB));
 #pragma unroll
@@ -114,6 +112,22 @@ __device__ __forceinline__ void rescale_chunk(const Chunk<F32IN>& d, const float
   }
 }
 
+// Warp -> (strip, row range): strip = warp % strips; warp k of a strip takes rows
+// [k * rpw, (k + 1) * rpw) clipped to the tokens (rpw: rows per warp, from the host)
+struct WarpWork {
+  int64_t col, row0, row1;
+};
+__device__ __forceinline__ WarpWork warp_work(const ActLaunch& A, int64_t rpw, int strips) {
+  const unsigned w = blockIdx.x * ACT_WARPS + threadIdx.x / 32;
+  const unsigned k = w / (unsigned)strips;
+  WarpWork ww;
+  ww.col = (int64_t)(w - k * (unsigned)strips) * STRIP + CHUNK * (threadIdx.x & 31);
+  ww.row0 = min((int64_t)k * rpw, A.tokens);
+  ww.row1 = min(ww.row0 + rpw, A.tokens);
+  return ww;
+}
+
+// largest |x| of a chunk (NaN if any is NaN), two independent chains
 __device__ __forceinline__ float absmax16(const float2 (&x)[8]) {
   float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
@@ -124,27 +138,12 @@ __device__ __forceinline__ float absmax16(const float2 (&x)[8]) {
   return max_nan(a0, a1);
 }
 
-// Warp -> (strip, row range): strip = warp % strips; the wps warps of a strip split the
-// rows evenly (ranges differ by at most one row)
-struct WarpWork {
-  int64_t col, row0, row1;
-};
-__device__ __forceinline__ WarpWork warp_work(const ActLaunch& A, int64_t wps, int strips) {
-  const int64_t w = (int64_t)blockIdx.x * ACT_WARPS + threadIdx.x / 32;
-  const int64_t k = w / strips;
-  WarpWork ww;
-  ww.col = (int64_t)(w % strips) * STRIP + CHUNK * (threadIdx.x & 31);
-  ww.row0 = (k < wps) ? (k * A.tokens) / wps : A.tokens;
-  ww.row1 = (k < wps) ? ((k + 1) * A.tokens) / wps : A.tokens;
-  return ww;
-}
-
 template <bool F32IN>
-__global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int strips) {
+__global__ void act_amax_kernel(const ActLaunch A, const int64_t rpw, const int strips) {
   // the quantization pass may start launching now; it waits for this grid's completion
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
-  const WarpWork ww = warp_work(A, wps, strips);
+  const WarpWork ww = warp_work(A, rpw, strips);
   const int64_t col = ww.col, row0 = ww.row0, row1 = ww.row1;
   const bool valid = col < A.n;
   float2 cv[8];
@@ -153,8 +152,13 @@ __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int 
   constexpr int RD = F32IN ? AMAX_RING / 2 : AMAX_RING;
   __shared__ __align__(16) uint4 ring_mem[ACT_WARPS][RD * 32 * LaneRing<F32IN, RD>::CB];
   const LaneRing<F32IN, RD> ring(ring_mem[threadIdx.x / 32], lane);
+  const int64_t step = A.ldx * (F32IN ? 4 : 2);
+  const char* src = reinterpret_cast<const char*>(A.X) + (row0 * A.ldx + col) * (F32IN ? 4 : 2);
 #pragma unroll
-  for (int j = 0; j < RD; ++j) ring.issue(A.X, row0 + j, A.ldx, col, valid && row0 + j < row1, j);
+  for (int j = 0; j < RD; ++j) {
+    ring.issue(src, valid && row0 + j < row1, j);
+    src += step;
+  }
   int slot = 0;
   for (int64_t row = row0; row < row1; ++row) {
     Chunk<F32IN> d;
@@ -162,7 +166,8 @@ __global__ void act_amax_kernel(const ActLaunch A, const int64_t wps, const int 
     if (!valid) zero_chunk<F32IN>(d);       // a lane past the last channel copied nothing
     float2 x[8];
     rescale_chunk<F32IN>(d, cv, x);        // the chunk is in registers: its slot is free
-    ring.issue(A.X, row + RD, A.ldx, col, valid && row + RD < row1, slot);
+    ring.issue(src, valid && row + RD < row1, slot);
+    src += step;
     a = max_nan(a, absmax16(x));
     slot = (slot + 1 == RD) ? 0 : slot + 1;
   }
@@ -202,7 +207,13 @@ __device__ __forceinline__ uint32_t e2m1x8_encode(const float2 (&y)[4]) {
 // -127..127): y = fl32(x * inv) clamped to [-Q, Q], then rounded to the nearest integer
 // (ties to even) by adding 1.5 * 2^23, whose last byte is then the integer's two's
 // complement. INT4: eight nibbles per word (value k in nibble k); INT8: four bytes per word.
-template <int ELEM>
+//
+// With a bf16 block scale s = bf16(fl32(a / Q)) (a the block's largest |x|), |x| / s stays
+// below Q / (1 - 2^-8) < Q + 1/2 (bf16 rounds with relative error at most 2^-8, and the binary32
+// roundings of 1/s and of the product move it by under 2^-22 relative), so the rounded code is
+// within [-Q, Q] without the clamp; CLAMP is needed for the E8M0 scales (a power of two can sit
+// up to a factor of 2 below a / Q).
+template <int ELEM, bool CLAMP>
 __device__ __forceinline__ void int_codes(const float2 (&x)[8], float2 iv, uint32_t (&w)[4]) {
   constexpr float Q = elem_qmax<ELEM>();
   const float2 magic = make_float2(12582912.0f, 12582912.0f), one = make_float2(1.0f, 1.0f);
@@ -210,8 +221,10 @@ __device__ __forceinline__ void int_codes(const float2 (&x)[8], float2 iv, uint3
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     float2 y = mul2(x[p], iv);
-    y.x = fminf(fmaxf(y.x, -Q), Q);
-    y.y = fminf(fmaxf(y.y, -Q), Q);
+    if constexpr (CLAMP) {
+      y.x = fminf(fmaxf(y.x, -Q), Q);
+      y.y = fminf(fmaxf(y.y, -Q), Q);
+    }
     const float2 z = fma2(y, one, magic);
     b[2 * p] = __float_as_uint(z.x);
     b[2 * p + 1] = __float_as_uint(z.y);
@@ -237,18 +250,18 @@ __device__ __forceinline__ void int_codes(const float2 (&x)[8], float2 iv, uint3
   }
 }
 
-template <int ELEM, int SCALE, int B, bool F32IN>
+template <int ELEM, int SCALE, int B, bool F32IN, bool SF_TC>
 __global__ void __launch_bounds__(ACT_WARPS * 32, 3)
-act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips, const int nparts) {
+act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const int nparts) {
   constexpr int LB = B / CHUNK;                   // lanes per block
   constexpr float QMAX = elem_qmax<ELEM>();
   constexpr int SCB = (SCALE == SCALE_BF16) ? 2 : 1;
   constexpr bool BYTE_CODES = (ELEM == ELEM_INT8);         // one code byte per element
   const int lane = threadIdx.x & 31;
-  const WarpWork ww = warp_work(A, wps, strips);
+  const WarpWork ww = warp_work(A, rpw, strips);
   const int64_t col = ww.col, row0 = ww.row0, row1 = ww.row1;
   const bool valid = col < A.n;
-  float s_t = 1.0f;
+  float s_t = 1.0f, is_t = 1.0f;
   // NVFP4: every E4M3 code's decoded scale fl32(s_t * e) and its reciprocal, per CTA
   __shared__ float2 tbl[SCALE == SCALE_E4M3 ? 128 : 1];
   if constexpr (SCALE == SCALE_E4M3) {
@@ -266,6 +279,7 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips, const i
 #pragma unroll
     for (int w = 0; w < ACT_WARPS; ++w) mx = max(mx, pmax[w]);
     s_t = nvfp4_tensor_scale(__uint_as_float(mx));
+    is_t = __frcp_rn(s_t);
     if (blockIdx.x == 0 && threadIdx.x == 0 && A.tensor_scale != nullptr) *A.tensor_scale = s_t;
     if (threadIdx.x < 128) {
       const uint32_t code = (threadIdx.x == 0 || threadIdx.x == 127) ? 1u : threadIdx.x;
@@ -284,27 +298,52 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips, const i
   constexpr int RD = F32IN ? QUANT_RING / 2 : QUANT_RING;
   __shared__ __align__(16) uint4 ring_mem[ACT_WARPS][RD * 32 * LaneRing<F32IN, RD>::CB];
   const LaneRing<F32IN, RD> ring(ring_mem[threadIdx.x / 32], lane);
+  // running addresses: the next row to copy, the code and scale destinations of this row
+  const int64_t step = A.ldx * (F32IN ? 4 : 2);
+  const char* src = reinterpret_cast<const char*>(A.X) + (row0 * A.ldx + col) * (F32IN ? 4 : 2);
 #pragma unroll
-  for (int j = 0; j < RD; ++j) ring.issue(A.X, row0 + j, A.ldx, col, valid && row0 + j < row1, j);
+  for (int j = 0; j < RD; ++j) {
+    ring.issue(src, valid && row0 + j < row1, j);
+    src += step;
+  }
+  uint8_t* qdst = A.x_packed + row0 * qpitch + (BYTE_CODES ? col : col / 2);
+  const int64_t b = col / B;
+  int64_t sidx = row0 * nb + b;
   int slot = 0;
-  for (int64_t row = row0; row < row1; ++row) {
+  for (int64_t row = row0; row < row1; ++row, qdst += qpitch, sidx += nb) {
+    // (a lane past the last channel copied nothing and computes on stale values: its block
+    // lies wholly past the last channel, and nothing of it is stored or flagged)
     Chunk<F32IN> cur;
     ring.read(slot, cur);
-    if (!valid) zero_chunk<F32IN>(cur);     // a lane past the last channel copied nothing
     float2 x[8];
     rescale_chunk<F32IN>(cur, cv, x);      // the chunk is in registers: its slot is free
-    ring.issue(A.X, row + RD, A.ldx, col, valid && row + RD < row1, slot);
+    ring.issue(src, valid && row + RD < row1, slot);
+    src += step;
     slot = (slot + 1 == RD) ? 0 : slot + 1;
     float a = absmax16(x);
-    bad |= !isfinite(a);
+    // (NVFP4: the pre-pass has flagged any non-finite x~ already)
+    if constexpr (SCALE != SCALE_E4M3) bad |= valid && !isfinite(a);
 #pragma unroll
     for (int off = 1; off < LB; off <<= 1) a = max_nan(a, __shfl_xor_sync(FULL, a, off));
     uint32_t code = 0;
     float inv = 0.0f;
     if (a > 0.0f) {
-      const ScaleVal sv = project_scale<SCALE>(div_qmax<(int)QMAX>(a), s_t, tbl);
-      code = sv.code;
-      inv = sv.ir;
+      const float v = div_qmax<(int)QMAX>(a);
+      if constexpr (SCALE == SCALE_E4M3) {
+        // E4M3 of fl32(v / s_t) through the reciprocal: v * fl32(1/s_t) lies within 3 ulps of
+        // the quotient, and E4M3 rounds (in its normal range) at the binary32 patterns whose
+        // low 20 bits are 0x80000; a product in [2^-6, 448) farther than 8 ulps from one
+        // rounds as the quotient does, anything else takes the division
+        const float u1 = v * is_t;
+        const uint32_t lo = __float_as_uint(u1) & 0xFFFFFu;
+        code = (u1 >= 0x1p-6f && u1 < 448.0f && (lo + 8u - 0x80000u) > 16u)
+                   ? e4m3_encode(u1) : project_code<SCALE>(v, s_t);
+        inv = tbl[code].y;
+      } else {
+        const ScaleVal sv = project_scale<SCALE>(v, s_t, tbl);
+        code = sv.code;
+        inv = sv.ir;
+      }
     }
     const float2 iv = make_float2(inv, inv);
     uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -318,41 +357,40 @@ act_quant_kernel(const ActLaunch A, const int64_t wps, const int strips, const i
         w[h] = e2m1x8_encode(y);
       }
     } else {
-      int_codes<ELEM>(x, iv, w);
+      int_codes<ELEM, SCALE != SCALE_BF16>(x, iv, w);
     }
     if (valid) {
       if (a == 0.0f) w[0] = w[1] = w[2] = w[3] = 0u;   // all-zero block: code 0 (also -0)
       if constexpr (BYTE_CODES) {
-        uint8_t* dst = A.x_packed + row * qpitch + col;
         if (wide) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(qdst) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
-          reinterpret_cast<uint2*>(dst)[0] = make_uint2(w[0], w[1]);
-          reinterpret_cast<uint2*>(dst)[1] = make_uint2(w[2], w[3]);
+          reinterpret_cast<uint2*>(qdst)[0] = make_uint2(w[0], w[1]);
+          reinterpret_cast<uint2*>(qdst)[1] = make_uint2(w[2], w[3]);
         }
       } else {
-        uint8_t* dst = A.x_packed + row * qpitch + col / 2;
         if (wide) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+          *reinterpret_cast<uint2*>(qdst) = make_uint2(w[0], w[1]);
         } else {
-          reinterpret_cast<uint32_t*>(dst)[0] = w[0];
-          reinterpret_cast<uint32_t*>(dst)[1] = w[1];
+          reinterpret_cast<uint32_t*>(qdst)[0] = w[0];
+          reinterpret_cast<uint32_t*>(qdst)[1] = w[1];
         }
       }
       if ((lane % LB) == 0) {
-        const int64_t b = col / B;
         if constexpr (SCB == 2) {
-          reinterpret_cast<uint16_t*>(A.scales)[row * nb + b] = (uint16_t)code;
+          reinterpret_cast<uint16_t*>(A.scales)[sidx] = (uint16_t)code;
         } else if constexpr (SCALE == SCALE_E4M3) {
           // the W4A4 GEMM's layout: [row / 128][n / 64][512 bytes], the four scales of a
           // 64-channel group of row r at (r % 32) * 16 + (r % 128 / 32) * 4
-          const int64_t r = row & 127;
-          const int64_t off = A.sf_tc ? ((row >> 7) * (A.n / 64) + (b >> 2)) * 512 +
-                                            (r & 31) * 16 + (r >> 5) * 4 + (b & 3)
-                                      : row * nb + b;
+          int64_t off = sidx;
+          if constexpr (SF_TC) {
+            const int64_t r = row & 127;
+            off = ((row >> 7) * (A.n / 64) + (b >> 2)) * 512 + (r & 31) * 16 + (r >> 5) * 4 +
+                  (b & 3);
+          }
           reinterpret_cast<uint8_t*>(A.scales)[off] = (uint8_t)code;
         } else {
-          reinterpret_cast<uint8_t*>(A.scales)[row * nb + b] = (uint8_t)code;
+          reinterpret_cast<uint8_t*>(A.scales)[sidx] = (uint8_t)code;
         }
       }
     }
@@ -376,33 +414,37 @@ int64_t resident_warps() {
   return warps;
 }
 
-// (strips x wps) warps: at most the resident warps (and cap_ctas CTAs), at least one row each
+// The grid of a pass: (strips x warps per strip), at most the resident warps (and cap_ctas
+// CTAs); rows per warp rpw = ceil(tokens / warps per strip), and only the warps with rows
+// are launched.
 struct RowGrid {
   int strips;
-  int64_t wps, ctas;
+  int64_t rpw, ctas;
 };
 template <auto KERNEL>
 RowGrid row_grid(const ActLaunch& A, int64_t cap_ctas) {
   RowGrid g;
   g.strips = (int)((A.n + STRIP - 1) / STRIP);
   const int64_t warps = std::min<int64_t>(resident_warps<KERNEL>(), cap_ctas * ACT_WARPS);
-  g.wps = std::max<int64_t>(1, std::min<int64_t>(warps / g.strips, A.tokens));
-  g.ctas = (g.wps * g.strips + ACT_WARPS - 1) / ACT_WARPS;
+  const int64_t wps = std::max<int64_t>(1, std::min<int64_t>(warps / g.strips, A.tokens));
+  g.rpw = std::max<int64_t>(1, (A.tokens + wps - 1) / wps);
+  const int64_t used = std::max<int64_t>(1, (A.tokens + g.rpw - 1) / g.rpw);
+  g.ctas = (used * g.strips + ACT_WARPS - 1) / ACT_WARPS;
   return g;
 }
 
-template <int ELEM, int SCALE, int B, bool F32IN>
+template <int ELEM, int SCALE, int B, bool F32IN, bool SF_TC>
 cudaError_t launch_fmt_dt(const ActLaunch& A, cudaStream_t s) {
-  constexpr auto QK = act_quant_kernel<ELEM, SCALE, B, F32IN>;
+  constexpr auto QK = act_quant_kernel<ELEM, SCALE, B, F32IN, SF_TC>;
   const RowGrid gq = row_grid<QK>(A, INT64_MAX / ACT_WARPS);
   if constexpr (SCALE != SCALE_E4M3) {
-    QK<<<(unsigned)gq.ctas, ACT_WARPS * 32, 0, s>>>(A, gq.wps, gq.strips, 0);
+    QK<<<(unsigned)gq.ctas, ACT_WARPS * 32, 0, s>>>(A, gq.rpw, gq.strips, 0);
     count_launches(1);
     return cudaGetLastError();
   } else {
     constexpr auto AK = act_amax_kernel<F32IN>;
     const RowGrid ga = row_grid<AK>(A, ACT_MAX_PARTS);
-    AK<<<(unsigned)ga.ctas, ACT_WARPS * 32, 0, s>>>(A, ga.wps, ga.strips);
+    AK<<<(unsigned)ga.ctas, ACT_WARPS * 32, 0, s>>>(A, ga.rpw, ga.strips);
     count_launches(1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -415,16 +457,25 @@ cudaError_t launch_fmt_dt(const ActLaunch& A, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, QK, A, gq.wps, gq.strips, (int)ga.ctas);
+    e = cudaLaunchKernelEx(&cfg, QK, A, gq.rpw, gq.strips, (int)ga.ctas);
     count_launches(1);
     return e;
   }
 }
 
+// the tensor core's scale layout exists for NVFP4 only
+template <int ELEM, int SCALE, int B, bool F32IN>
+cudaError_t launch_layout(const ActLaunch& A, cudaStream_t s) {
+  if constexpr (SCALE == SCALE_E4M3) {
+    if (A.sf_tc) return launch_fmt_dt<ELEM, SCALE, B, F32IN, true>(A, s);
+  }
+  return launch_fmt_dt<ELEM, SCALE, B, F32IN, false>(A, s);
+}
+
 template <int ELEM, int SCALE, int B>
 cudaError_t launch_fmt(const ActLaunch& A, int esize, cudaStream_t s) {
-  return (esize == 4) ? launch_fmt_dt<ELEM, SCALE, B, true>(A, s)
-                      : launch_fmt_dt<ELEM, SCALE, B, false>(A, s);
+  return (esize == 4) ? launch_layout<ELEM, SCALE, B, true>(A, s)
+                      : launch_layout<ELEM, SCALE, B, false>(A, s);
 }
 
 }  // namespace

@@ -1,4 +1,4 @@
-"""The binary32 block sums of the bf16-scale r-step, checked against their error bound (host).
+"""Two shortcuts the kernels take with bf16 block scales, checked against their bounds (host).
 
 The solve kernel's r-step for the bf16-scale formats (INT4, INT8) forms the least-squares
 quotient num/den of a block in binary32 first: each lane accumulates its 16 elements as two
@@ -94,3 +94,18 @@ def test_binary32_block_sums_within_bound(B, qmax, kind):
     exact32 = v.astype(F64).astype(F32)
     assert np.array_equal(_bf16_rn(v32)[sure], _bf16_rn(exact32)[sure])
     assert sure.mean() > 0.99
+
+
+@pytest.mark.parametrize("Q", [7, 127])
+def test_bf16_scale_codes_stay_in_range_without_a_clamp(Q):
+    """The activation quantizer rounds x * fl32(1/s) to an integer code without clamping it when
+    s is a bf16 block scale bf16(fl32(a/Q)), a the block's largest |x|: the quotient stays below
+    Q + 1/2. Checked for every binary32 a in [1, 2) (the ratio repeats in every binade above
+    the bf16 scale's lower clamp, which only makes s larger)."""
+    a = np.arange(0x3F800000, 0x40000000, dtype=np.uint64).astype(np.uint32).view(F32)
+    v = (a.astype(F64) / Q).astype(F32)
+    u = v.view(np.uint32).astype(np.uint64)
+    s = (((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16).astype(np.uint32).view(F32)
+    inv = (1.0 / s.astype(F64)).astype(F32)
+    y = (a.astype(F64) * inv.astype(F64)).astype(F32)
+    assert float(y.max()) < Q + 0.5
