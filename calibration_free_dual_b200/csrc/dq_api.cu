@@ -232,6 +232,7 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
       L.upd_c = update != DQ_UPDATE_ROW_ONLY;
       L.qch = qch;
       L.err_word = errp;
+      L.tma = 1;     // cleared when a map cannot be made: the kernel then copies per thread
       for (int k = 0; k < c; ++k) {
         const int64_t idx = grp[base + k];
         const dq_matrix& d = mats[idx];
@@ -251,6 +252,8 @@ dq_status dq_solve_batched_ex(const dq_matrix* mats, int64_t count, int32_t dtyp
         sm.ws_wsq = slots[idx].wsq;
         sm.ws_qch = slots[idx].qch;
         sm.amax_bits = slots[idx].amax;
+        if (L.tma && !dq::make_w_map(&L.wmap[k], d.W, ms[i], ns[i], d.ldw, esize, plan.S))
+          L.tma = 0;
       }
       if (fmt.kind == DQ_NVFP4) {
         if ((st = from_cuda(dq::launch_solve_amax(L, c, esize, s))) != DQ_OK) return st;

@@ -495,6 +495,26 @@ int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+// W as [m][n/16][16] (rows, 16-column pieces, columns), box {16, S, solve_box_rows(S)}: a box
+// is S pieces of solve_box_rows(S) rows, laid out row-major with the 32-byte (bf16) or 64-byte
+// (fp32) swizzle, i.e. 16-byte chunk h of piece P at chunk 2P + (h ^ bit 2 of P), resp.
+// 4P + (h ^ bits 1-2 of P): the order in which the solve kernel reads its resident rows.
+// Rows past m read as zero.
+bool make_w_map(CUtensorMap* map, const void* W, int64_t m, int64_t n, int64_t ldw, int esize,
+                int S) {
+  EncodeTiledFn fn = encoder();
+  if (fn == nullptr || (esize != 2 && esize != 4) || n % 16 != 0) return false;
+  const cuuint64_t dims[3] = {16, (cuuint64_t)(n / 16), (cuuint64_t)m};
+  const cuuint64_t strides[2] = {(cuuint64_t)(16 * esize), (cuuint64_t)(ldw * esize)};
+  const cuuint32_t box[3] = {16, (cuuint32_t)S, (cuuint32_t)solve_box_rows(S)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32, 3,
+            const_cast<void*>(W), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            esize == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t K, bool sfa_given) {
   // interleaved scale factors, rows padded to whole 128-row blocks
   return (size_t)((sfa_given ? 0 : round_up(T, BM)) + round_up(N, BN)) * (size_t)(K / 16) + 256;

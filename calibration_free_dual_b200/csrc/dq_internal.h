@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>   // CUtensorMap (the encoder is fetched from the driver at run time)
 #include <cuda_runtime.h>
 
 namespace dq {
@@ -36,7 +37,21 @@ struct SolveLaunch {
   int qch;                     // extended kernel: record the Q-change trace
   unsigned* err_word;
   SolveMat mats[SOLVE_MAXMATS];
+  // tma != 0: wmap[i] maps matrix i's W as [m][n/16][16] (rows, 16-column pieces, columns)
+  // with boxes of {16, S, solve_box_rows(S)} and the 32-byte (bf16) or 64-byte (fp32)
+  // swizzle, and the kernel copies its resident rows with the tensor memory accelerator
+  int tma;
+  CUtensorMap wmap[SOLVE_MAXMATS];
 };
+
+// rows per tensor-map box of the solve's resident-row copy: one sweep (512/S rows), at most
+// the 256 a box dimension allows
+__host__ __device__ constexpr int solve_box_rows(int S) { return SOLVE_NT / S < 256 ? SOLVE_NT / S : 256; }
+
+// the solve's W tensor map (see SolveLaunch::wmap); false when the driver's encoder is missing
+// or refuses the shape
+bool make_w_map(CUtensorMap* map, const void* W, int64_t m, int64_t n, int64_t ldw, int esize,
+                int S);
 
 struct SolvePlan {
   int S;        // 16-column pieces per CTA tile (tile width TN = 16*S)
@@ -51,7 +66,7 @@ struct SolvePlan {
 // the per-warp column partials and the per-warp fp64 error sums; with the Q-change trace
 // also the previous iteration's scale codes, its 1/c and per-warp Q-change sums.
 struct SolveSmem {
-  size_t w, codes, tbl, cvec, icvec, red, cols, pcodes, picvec, qred, total;
+  size_t w, codes, tbl, cvec, icvec, red, cols, pcodes, picvec, qred, bar, total;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -72,6 +87,7 @@ __host__ __device__ inline SolveSmem solve_smem(int m, int R, int S, int LPB, in
   l.pcodes = off; if (qch) off = align_up(off + mpad * NBLK * scb, 16);
   l.picvec = off; if (qch) off = align_up(off + TN * 4, 16);
   l.qred = off;   if (qch) off = align_up(off + (size_t)NWARP * 2 * 8, 16);
+  l.bar = off;    off = align_up(off + 8, 16);           // the resident-row copy's mbarrier
   l.total = off;
   return l;
 }

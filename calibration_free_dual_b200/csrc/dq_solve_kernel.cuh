@@ -12,9 +12,10 @@
 // TN = 16*S columns and ALL m rows of it, so every reduction of the solve is CTA-local and
 // needs only __syncthreads:
 //   * the first R rows of the tile stay in shared memory for the whole solve (copied once
-//     from HBM); the remaining rows are read again from L2 on every pass with 256-bit loads
-//     marked evict-last (the streamed rows of all resident CTAs stay far below the 126 MB
-//     L2), the next row in flight while the current one is processed;
+//     from HBM by the tensor memory accelerator: tensor-map boxes whose swizzle is the row
+//     loop's bank-conflict-free order); the remaining rows are read again from L2 on every
+//     pass with 256-bit loads marked evict-last (the streamed rows of all resident CTAs stay
+//     far below the 126 MB L2), the next row in flight while the current one is processed;
 //   * each thread owns one 16-column piece of a set of rows; LPB = B/16 neighbouring lanes
 //     share one format block and combine its r-step sums with xor shuffles;
 //   * Q-, r- and c-step run per row in registers with packed fp32x2 arithmetic
@@ -37,6 +38,36 @@ namespace {
 
 constexpr unsigned FULL = 0xFFFFFFFFu;
 constexpr int NWARP = SOLVE_NT / 32;
+
+// ---- the resident-row copy by the tensor memory accelerator: boxes of the W tensor map
+// land in shared memory and complete on one mbarrier (transaction bytes)
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void tma_box_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                           int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];"
+      :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+// bounded wait for phase 0 of the copy's mbarrier: false after 2 s of global time
+__device__ __forceinline__ bool copy_wait(uint32_t bar) {
+  uint64_t t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar) : "memory");
+    if (ok) return true;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 > 2000000000ull) return false;
+  }
+}
 
 // 16-byte chunk position of chunk h of piece P (the 16 columns one thread owns in one row;
 // row-major [R][TN] tile, CPP chunks per piece). The 8 lanes of a quarter warp read 8
@@ -195,20 +226,43 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     else reinterpret_cast<uint8_t*>(pcodes_v)[code0 + k * (NT / LPB)] = (uint8_t)code;
   };
 
-  // ---- rows [0, R) into shared memory (their only read from HBM) by asynchronous 16-byte
-  // copies, all in flight at once; rows past m (only in the last sweep) are zero-filled and
-  // add nothing to any sum. Issued first, awaited before the first pass; the iteration-0
-  // pass checks every row for non-finite values.
-  {
+  // ---- rows [0, R) into shared memory (their only read from HBM), all in flight at once;
+  // rows past m (only in the last sweep) are zero-filled and add nothing to any sum. With a
+  // tensor map of W, one thread issues boxes of {16 columns, S pieces, BR rows} through the
+  // tensor memory accelerator: the map's 32-byte (bf16) / 64-byte (fp32) swizzle puts every
+  // 16-byte chunk where chunk_pos places it (the swizzle works on address bits, so the copy
+  // needs the buffer aligned to the swizzle's 256- / 512-byte period). Otherwise every thread
+  // issues asynchronous 16-byte copies. Awaited before the first pass; the iteration-0 pass
+  // checks every row for non-finite values.
+  const uint32_t wsm_addr = smem_addr(Wsm);
+  const uint32_t wbar = smem_addr(smem + lay.bar);
+  const bool tma = L.tma != 0 && L.R > 0 && (wsm_addr & (ESZ == 2 ? 255u : 511u)) == 0;
+  if (tma) {
+    // boxes that start below m (a box that runs past m is zero-filled beyond it); the rows of
+    // boxes wholly past m (a 512-row sweep takes two boxes when S = 1) are zeroed here
+    constexpr int BR = solve_box_rows(S);
+    const int rtma = min(L.R, (m + BR - 1) / BR * BR);
+    if (tid == 0) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(wbar) : "memory");
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                   :: "r"(wbar), "r"((uint32_t)rtma * TN * ESZ) : "memory");
+      for (int r0 = 0; r0 < rtma; r0 += BR)
+        tma_box_3d(wsm_addr + (uint32_t)r0 * TN * ESZ, &L.wmap[blockIdx.y], 0, tile * S, r0,
+                   wbar);
+    }
+    uint4* zw = reinterpret_cast<uint4*>(Wsm + (size_t)rtma * TN * ESZ);
+    for (int i = tid; i < (L.R - rtma) * TN * ESZ / 16; i += NT) zw[i] = make_uint4(0u, 0u, 0u, 0u);
+  } else {
     constexpr int CH = TN * ESZ / 16;      // 16-byte chunks per row
     const char* base = reinterpret_cast<const char*>(M.W) + (int64_t)col0 * ESZ;
-    const uint32_t dst0 = static_cast<uint32_t>(__cvta_generic_to_shared(Wsm));
 #pragma unroll 4
     for (int ch = tid; ch < L.R * CH; ch += NT) {
       const int row = ch / CH, part = ch % CH;
       const bool in = row < m;
       const char* src = base + (int64_t)(in ? row : 0) * pitch + part * 16;
-      const uint32_t dst = dst0 + 16u * chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ);
+      const uint32_t dst = wsm_addr + 16u * chunk_pos<ESZ>(row * S + part / ESZ, part % ESZ);
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                    :: "r"(dst), "l"(src), "r"(in ? 16 : 0) : "memory");
     }
@@ -245,8 +299,18 @@ solve_kernel(const __grid_constant__ SolveLaunch L) {
     icvec[tid] = __frcp_rn(cj);
   }
 
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
+  if (tma) {
+    // (the barrier's initialisation is visible to all threads after this sync)
+    __syncthreads();
+    const bool ok = copy_wait(wbar);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) atomicOr(L.err_word, ERRBIT_TIMEOUT);
+      return;
+    }
+  } else {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+  }
 
   float2 cc[8], ic[8];
   auto load_c = [&]() {
