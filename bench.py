@@ -788,7 +788,13 @@ def run_ours(args, world, rank, local):
                         kernel_ms_per_step=kms_step, launches_timed=timer.used,
                         traffic_unit="DRAM bytes per solve launch (ncu capture of the same "
                                      "kernel source, layer-set average), null if the kernel "
-                                     "changed since")
+                                     "changed since",
+                        note="achieved = the algorithmic bytes of a per-iteration streaming "
+                             "solve (W and the block-scale state every iteration, the codes "
+                             "once) over the kernel time; the kernel itself reads W from HBM "
+                             "about once per solve (dram_gbs_measured)")
+    if traffic is not None:
+        roof["dram_gbs_measured"] = traffic * per_step / (kms_step * 1e-3) / 1e9
     act_bpe = ACT_BYTES_PER_ELEM.get(args.fmt if args.fmt != "INT4_G64" else "INT4")
     act_elems = X.numel()
     step_bytes = (bpe + prepass_bytes_per_elem(args.fmt)) * elems + (act_bpe or 0) * act_elems
