@@ -659,7 +659,7 @@ def run_ours(args, world, rank, local):
     fmt = dq.fmt_of(args.fmt)
     headline = args.fmt == "NVFP4" and args.update == "both" and not args.qchange
     stream = torch.cuda.current_stream(dev)
-    split = args.split and world > 1
+    split = bool(args.split)          # (one rank: the whole layer set, the same work either way)
     if split:
         # one layer set shared by the ranks, matrices assigned by element count
         sizes = [m * n for _, _, m, n in full_layer]
