@@ -8,9 +8,10 @@ activation with the column scales of that step's block-0 k_proj (dq_act_quant).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--split]
 
 The JSON line also carries, measured in the same run on one GPU: the activation quantizer
-alone (NVFP4 and INT4 g=128, L2 flushed, SQNR with and without c), the Llama-3.2-1B-shaped
-MXFP4 and Llama-2-7B-shaped MXINT4 layer sets in their own shapes, and the convergence of
-block 0 of the three layer sets (the Q-change trace and the normalised MSE).
+alone (NVFP4 and INT4 g=128, calls back to back over inputs larger than L2 and one call behind
+an L2 flush, SQNR with and without c), the Llama-3.2-1B-shaped MXFP4 and Llama-2-7B-shaped
+MXINT4 layer sets in their own shapes, and the convergence of block 0 of the three layer sets
+(the Q-change trace and the normalised MSE).
 
 Other measurements (same JSON conventions): --fmt/--update/--qchange (other formats and the
 ablation modes of the headline step), --act (the activation quantizer alone), --gemm (the
