@@ -14,7 +14,8 @@
 // 16 column scales in registers for all its rows and walks down the rows, so a warp's loads,
 // its 8-byte code stores and its scale stores are contiguous and c is read once per warp.
 // Rows arrive through a per-lane ring of asynchronous copies in shared memory (several rows
-// in flight, no registers held). A block of B channels spans B/16 lanes, which combine their
+// in flight, no registers held); the quantization pass works on two rows at a time (two
+// independent chains). A block of B channels spans B/16 lanes, which combine their
 // absolute maxima with xor shuffles; the block scale is computed once per 16 elements. NVFP4
 // needs the global amax of x~ first: a separate pass over the same rows that writes one
 // maximum per CTA (no atomics, nothing to clear beforehand); the quantization pass is launched
@@ -251,7 +252,7 @@ __device__ __forceinline__ void int_codes(const float2 (&x)[8], float2 iv, uint3
 }
 
 template <int ELEM, int SCALE, int B, bool F32IN, bool SF_TC>
-__global__ void __launch_bounds__(ACT_WARPS * 32, 3)
+__global__ void __launch_bounds__(ACT_WARPS * 32, 2)
 act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const int nparts) {
   constexpr int LB = B / CHUNK;                   // lanes per block
   constexpr float QMAX = elem_qmax<ELEM>();
@@ -310,22 +311,25 @@ act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const i
   const int64_t b = col / B;
   int64_t sidx = row0 * nb + b;
   int slot = 0;
-  for (int64_t row = row0; row < row1; ++row, qdst += qpitch, sidx += nb) {
+  // one row's chunk from the ring (the next row of the lane's range is then put in flight)
+  auto load_row = [&](int64_t row, float2 (&x)[8]) {
     // (a lane past the last channel copied nothing and computes on stale values: its block
     // lies wholly past the last channel, and nothing of it is stored or flagged)
     Chunk<F32IN> cur;
     ring.read(slot, cur);
-    float2 x[8];
     rescale_chunk<F32IN>(cur, cv, x);      // the chunk is in registers: its slot is free
     ring.issue(src, valid && row + RD < row1, slot);
     src += step;
     slot = (slot + 1 == RD) ? 0 : slot + 1;
-    float a = absmax16(x);
+  };
+  // the block maximum, scale code, reciprocal and element codes of one row
+  auto quant_row = [&](const float2 (&x)[8], float& a, uint32_t& code, uint32_t (&w)[4]) {
+    a = absmax16(x);
     // (NVFP4: the pre-pass has flagged any non-finite x~ already)
     if constexpr (SCALE != SCALE_E4M3) bad |= valid && !isfinite(a);
 #pragma unroll
     for (int off = 1; off < LB; off <<= 1) a = max_nan(a, __shfl_xor_sync(FULL, a, off));
-    uint32_t code = 0;
+    code = 0;
     float inv = 0.0f;
     if (a > 0.0f) {
       const float v = div_qmax<(int)QMAX>(a);
@@ -346,7 +350,7 @@ act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const i
       }
     }
     const float2 iv = make_float2(inv, inv);
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    w[0] = w[1] = w[2] = w[3] = 0u;
     if constexpr (ELEM == ELEM_E2M1) {
       // four conversions straight into the bytes of one word
 #pragma unroll
@@ -359,6 +363,10 @@ act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const i
     } else {
       int_codes<ELEM, SCALE != SCALE_BF16>(x, iv, w);
     }
+  };
+  // the row's codes and scale code (blocks of a lane past the last channel: nothing)
+  auto store_row = [&](int64_t row, uint8_t* qdst, int64_t sidx, float a, uint32_t code,
+                       uint32_t (&w)[4]) {
     if (valid) {
       if (a == 0.0f) w[0] = w[1] = w[2] = w[3] = 0u;   // all-zero block: code 0 (also -0)
       if constexpr (BYTE_CODES) {
@@ -394,6 +402,27 @@ act_quant_kernel(const ActLaunch A, const int64_t rpw, const int strips, const i
         }
       }
     }
+  };
+  // two rows per iteration: two independent chains for the scheduler to interleave
+  int64_t row = row0;
+  for (; row + 1 < row1; row += 2, qdst += 2 * qpitch, sidx += 2 * nb) {
+    float2 x0[8], x1[8];
+    load_row(row, x0);
+    load_row(row + 1, x1);
+    float a0, a1;
+    uint32_t c0, c1, w0[4], w1[4];
+    quant_row(x0, a0, c0, w0);
+    quant_row(x1, a1, c1, w1);
+    store_row(row, qdst, sidx, a0, c0, w0);
+    store_row(row + 1, qdst + qpitch, sidx + nb, a1, c1, w1);
+  }
+  if (row < row1) {
+    float2 x0[8];
+    load_row(row, x0);
+    float a0;
+    uint32_t c0, w0[4];
+    quant_row(x0, a0, c0, w0);
+    store_row(row, qdst, sidx, a0, c0, w0);
   }
   if (bad) atomicOr(A.err_word, ERRBIT_NONFINITE);
 }
